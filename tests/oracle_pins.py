@@ -1,0 +1,358 @@
+"""Pins for the float64 oracle, each against something other than the orc.
+
+Sources of the pins: closed forms, invariants of softmax attention, a library
+routine (torch's float64 math SDPA), brute force over tiny inputs in exact
+summation, and the pages' own claims (the online recurrence of the MCU page's
+§二 equals the two-pass softmax exactly; causal row 0 sees only key 0; GQA
+shares one K/V head across a group of query heads).
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+
+RNG = np.random.default_rng(1234)
+
+
+def rand(*shape, rng=RNG):
+    return rng.standard_normal(shape)
+
+
+def brute_force(q, k, v, scale, causal, lens):
+    """Scalar loops with math.fsum: one row at a time, no vectorised code."""
+    B, Hq, N, d = q.shape
+    Hk = k.shape[1]
+    G = Hq // Hk
+    o = np.zeros((B, Hq, N, v.shape[3]))
+    lse = np.full((B, Hq, N), -math.inf)
+    for b in range(B):
+        L = N if lens is None else min(max(int(lens[b]), 0), N)
+        for h in range(Hq):
+            kh = h // G
+            for i in range(N):
+                keys = [j for j in range(N) if j < L and (not causal or j <= i)]
+                if not keys:
+                    continue
+                s = {j: scale * math.fsum(q[b, h, i, c] * k[b, kh, j, c] for c in range(d))
+                     for j in keys}
+                mx = max(s.values())
+                w = {j: math.exp(s[j] - mx) for j in keys}
+                tot = math.fsum(w.values())
+                for c in range(v.shape[3]):
+                    o[b, h, i, c] = math.fsum(w[j] * v[b, kh, j, c] for j in keys) / tot
+                lse[b, h, i] = mx + math.log(tot)
+    return o, lse
+
+
+def close(a, b, tol=1e-12):
+    a, b = np.asarray(a), np.asarray(b)
+    fin = np.isfinite(b)
+    assert np.array_equal(np.isfinite(a), fin)
+    assert np.array_equal(a[~fin], b[~fin])
+    if fin.any():
+        assert np.max(np.abs(a[fin] - b[fin])) <= tol * max(1.0, np.max(np.abs(b[fin])))
+
+
+# ---------------------------------------------------------------- brute force
+
+def pin_matches_scalar_brute_force(orc):
+    q, k, v = rand(2, 4, 6, 3), rand(2, 2, 6, 3), rand(2, 2, 6, 2)
+    for causal, lens in itertools.product([False, True], [None, [3, 0]]):
+        o, lse = orc.attention(q, k, v, 0.7, causal, lens)
+        ob, lseb = brute_force(q, k, v, 0.7, causal, lens)
+        close(o, ob)
+        close(lse, lseb)
+
+
+# ------------------------------------------------------------ library routine
+
+def pin_matches_torch_math_sdpa(orc):
+    for causal, G in itertools.product([False, True], [1, 2, 4]):
+        _sdpa_case(orc, causal, G)
+
+
+def _sdpa_case(orc, causal, G):
+    B, Hk, N, d = 2, 2, 37, 16
+    Hq = Hk * G
+    q, k, v = rand(B, Hq, N, d), rand(B, Hk, N, d), rand(B, Hk, N, d)
+    lens = [37, 20]
+    scale = 0.3
+    o, _ = orc.attention(q, k, v, scale, causal, lens)
+    i = torch.arange(N)[:, None]
+    j = torch.arange(N)[None, :]
+    mask = torch.stack([(j < L) & ((j <= i) if causal else torch.ones_like(j <= i))
+                        for L in lens])[:, None]
+    kt = torch.from_numpy(k).repeat_interleave(G, dim=1)
+    vt = torch.from_numpy(v).repeat_interleave(G, dim=1)
+    with torch.nn.attention.sdpa_kernel(torch.nn.attention.SDPBackend.MATH):
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q), kt, vt, attn_mask=mask, scale=scale).numpy()
+    close(o, ref, 1e-12)
+
+
+# ------------------------------------------------- recurrence == two-pass ([MCU] §二)
+
+def pin_online_recurrence_equals_two_pass_all_tilings(orc):
+    for fn in (orc.online_attention_flowchart, orc.online_attention_equations):
+        _all_tilings(orc, fn)
+
+
+def _all_tilings(orc, fn):
+    rng = np.random.default_rng(7)
+    N, d = 7, 3
+    q, k, v = rng.standard_normal((1, 2, N, d)), rng.standard_normal((1, 1, N, d)), \
+        rng.standard_normal((1, 1, N, 2))
+    for causal, lens in [(False, None), (True, None), (False, [4]), (True, [5]), (False, [0])]:
+        ref_o, ref_l = orc.attention(q, k, v, 1.3, causal, lens)
+        for tr, tc in itertools.product(range(1, N + 1), repeat=2):
+            o, l = fn(q, k, v, 1.3, causal, lens, tile_r=tr, tile_c=tc)
+            close(o, ref_o, 1e-12)
+            close(l, ref_l, 1e-12)
+
+
+def pin_online_recurrence_adversarial_scores(orc):
+    """Increasing, decreasing and ±30-spread scores force every rescale branch."""
+    for fn in (orc.online_attention_flowchart, orc.online_attention_equations):
+        _adversarial(orc, fn)
+
+
+def _adversarial(orc, fn):
+    N = 9
+    v = RNG.standard_normal((1, 1, N, 3))
+    k = np.zeros((1, 1, N, 1))
+    q = np.ones((1, 1, N, 1))
+    for keys in [np.arange(N) * 4.0, -np.arange(N) * 4.0, np.array([30, -30] * 4 + [0.0])]:
+        k[0, 0, :, 0] = keys
+        ref_o, ref_l = orc.attention(q, k, v, 1.0, False, None)
+        for tc in range(1, N + 1):
+            o, l = fn(q, k, v, 1.0, False, None, tile_r=N, tile_c=tc)
+            close(o, ref_o, 1e-12)
+            close(l, ref_l, 1e-12)
+
+
+# ------------------------------------------------------------------ invariants
+
+def pin_softmax_rows_sum_to_one_and_are_nonnegative(orc):
+    q, k = rand(5, 8), rand(9, 8)
+    for causal, L in [(False, 9), (True, 9), (False, 4), (True, 2)]:
+        ok = orc.allowed_keys(np.arange(5), 9, causal, L)
+        p, m, l = orc.two_pass_softmax(orc.scores(q, k, 0.5, ok))
+        w = p / l[:, None]
+        assert np.all(w >= 0)
+        assert np.all(w[~ok] == 0)
+        assert np.max(np.abs(w.sum(axis=1) - 1.0)) < 1e-12
+        assert np.max(p) == 1.0  # the row max contributes exp(0)
+
+
+def pin_uniform_v_returns_v(orc):
+    q, k = rand(1, 3, 11, 4) * 5, rand(1, 3, 11, 4) * 5
+    c = rand(4)
+    v = np.broadcast_to(c, (1, 3, 11, 4)).copy()
+    for causal in (False, True):
+        o, _ = orc.attention(q, k, v, 1.0, causal, [7])
+        close(o, np.broadcast_to(c, o.shape), 1e-13)
+
+
+def pin_one_hot_score_selects_v_row(orc):
+    """Row i scores key t(i) at 60 and every other key at 0: O_i = V_t(i) within e^-60."""
+    N = 10
+    v = rand(1, 1, N, 5)
+    target = RNG.permutation(N)
+    k = np.eye(N)[None, None] * 60.0
+    q = np.zeros((1, 1, N, N))
+    q[0, 0, np.arange(N), target] = 1.0
+    o, lse = orc.attention(q, k, v, 1.0, False, None)
+    assert np.max(np.abs(o[0, 0] - v[0, 0, target])) < 1e-14
+    assert np.max(np.abs(lse[0, 0] - 60.0)) < 1e-12
+
+
+def pin_single_allowed_key_is_exact(orc):
+    """Key padding to one key: O_i = V_0 and LSE_i = s_i0, exactly."""
+    q, k, v = rand(1, 2, 8, 4), rand(1, 1, 8, 4), rand(1, 1, 8, 4)
+    o, lse = orc.attention(q, k, v, 0.9, False, [1])
+    assert np.array_equal(o[0], np.broadcast_to(v[0, 0, 0], (2, 8, 4)))
+    s0 = 0.9 * (q[0, :, :, :] @ k[0, 0, 0])
+    assert np.max(np.abs(lse[0] - s0)) < 1e-15 * 8
+
+
+def pin_causal_row0_is_v0_and_future_keys_do_not_matter(orc):
+    q, k, v = rand(1, 1, 12, 4), rand(1, 1, 12, 4), rand(1, 1, 12, 3)
+    o, lse = orc.attention(q, k, v, 0.8, True, None)
+    assert np.array_equal(o[0, 0, 0], v[0, 0, 0])
+    assert lse[0, 0, 0] == 0.8 * (q[0, 0, 0] @ k[0, 0, 0])
+    for i in range(12):
+        k2, v2 = k.copy(), v.copy()
+        k2[0, 0, i + 1:] = rand(12 - i - 1, 4) * 9
+        v2[0, 0, i + 1:] = rand(12 - i - 1, 3) * 9
+        o2, lse2 = orc.attention(q, k2, v2, 0.8, True, None)
+        assert np.array_equal(o2[0, 0, : i + 1], o[0, 0, : i + 1])
+        assert np.array_equal(lse2[0, 0, : i + 1], lse[0, 0, : i + 1])
+
+
+def pin_scale_zero_closed_form(orc):
+    """scale = 0: O_i is the mean of the allowed V rows and LSE_i = ln(#allowed)."""
+    N = 9
+    q, k, v = rand(1, 1, N, 4), rand(1, 1, N, 4), rand(1, 1, N, 3)
+    for causal, L in [(False, N), (True, N), (False, 5), (True, 4)]:
+        o, lse = orc.attention(q, k, v, 0.0, causal, [L])
+        for i in range(N):
+            n_ok = min(L, i + 1) if causal else L
+            assert np.max(np.abs(o[0, 0, i] - v[0, 0, :n_ok].mean(axis=0))) < 1e-14
+            assert abs(lse[0, 0, i] - math.log(n_ok)) < 1e-14
+
+
+def pin_shift_of_row_scores(orc):
+    """Adding c to every score of a row leaves O and shifts LSE by c.
+
+    The shift is built into the inputs: an extra feature 1 on every key and c/scale
+    on every query, so the oracle sees an ordinary (d+1)-wide problem.
+    """
+    N, d, scale = 10, 4, 0.6
+    q, k, v = rand(1, 2, N, d), rand(1, 1, N, d), rand(1, 1, N, 3)
+    c = rand(1, 2, N, 1) * 7
+    q2 = np.concatenate([q, c / scale], axis=3)
+    k2 = np.concatenate([k, np.ones((1, 1, N, 1))], axis=3)
+    for causal, lens in [(False, None), (True, [6])]:
+        o, lse = orc.attention(q, k, v, scale, causal, lens)
+        o2, lse2 = orc.attention(q2, k2, v, scale, causal, lens)
+        close(o2, o, 1e-12)
+        close(lse2, lse + c[..., 0], 1e-12)
+
+
+def pin_permutations(orc):
+    N = 11
+    q, k, v = rand(1, 1, N, 4), rand(1, 1, N, 4), rand(1, 1, N, 3)
+    o, lse = orc.attention(q, k, v, 0.5, False, None)
+    perm = RNG.permutation(N)
+    o2, lse2 = orc.attention(q, k[:, :, perm], v[:, :, perm], 0.5, False, None)
+    close(o2, o, 1e-12)
+    close(lse2, lse, 1e-12)
+    o3, lse3 = orc.attention(q[:, :, perm], k, v, 0.5, False, None)
+    close(o3, o[:, :, perm], 1e-12)
+    close(lse3, lse[:, :, perm], 1e-12)
+
+
+def pin_gqa_equals_mha_on_repeated_kv(orc):
+    for Hq, Hk in [(4, 2), (8, 2), (6, 1), (4, 4)]:
+        _gqa_case(orc, Hq, Hk)
+
+
+def _gqa_case(orc, Hq, Hk):
+    q, k, v = rand(2, Hq, 9, 4), rand(2, Hk, 9, 4), rand(2, Hk, 9, 4)
+    G = Hq // Hk
+    for causal in (False, True):
+        o, lse = orc.attention(q, k, v, 0.7, causal, [9, 5])
+        o2, lse2 = orc.attention(q, np.repeat(k, G, axis=1), np.repeat(v, G, axis=1),
+                                    0.7, causal, [9, 5])
+        close(o, o2, 0)
+        close(lse, lse2, 0)
+
+
+def pin_n_equals_one(orc):
+    q, k, v = rand(1, 3, 1, 8), rand(1, 3, 1, 8), rand(1, 3, 1, 8)
+    for causal in (False, True):
+        o, lse = orc.attention(q, k, v, 0.4, causal, None)
+        assert np.array_equal(o, v)
+        assert np.max(np.abs(lse[..., 0] - 0.4 * np.einsum("hd,hd->h", q[0, :, 0], k[0, :, 0]))) \
+            < 1e-15 * 8
+
+
+def pin_key_padding_equals_truncated_keys(orc):
+    N, L = 12, 7
+    q, k, v = rand(1, 2, N, 4), rand(1, 2, N, 4), rand(1, 2, N, 3)
+    for causal in (False, True):
+        o, lse = orc.attention(q, k, v, 0.5, causal, [L])
+        # rows < L with truncated K/V of length L: an independent smaller problem
+        o2, lse2 = orc.attention(q[:, :, :L], k[:, :, :L], v[:, :, :L], 0.5, causal, None)
+        close(o[:, :, :L], o2, 1e-12)
+        close(lse[:, :, :L], lse2, 1e-12)
+        if not causal:
+            # rows >= L see the same L keys; a row's output is that of the row alone
+            for i in range(L, N):
+                o3, _ = orc.attention(q[:, :, i:i + 1], k[:, :, :L], v[:, :, :L], 0.5, False, None)
+                close(o[:, :, i:i + 1], o3, 1e-12)
+
+
+def pin_empty_rows(orc):
+    q, k, v = rand(2, 2, 5, 4), rand(2, 1, 5, 4), rand(2, 1, 5, 4)
+    o, lse = orc.attention(q, k, v, 0.5, True, [0, 5])
+    assert np.all(o[0] == 0) and np.all(np.isneginf(lse[0]))
+    assert np.all(np.isfinite(lse[1]))
+    for fn in (orc.online_attention_flowchart, orc.online_attention_equations):
+        o2, lse2 = fn(q, k, v, 0.5, True, [0, 5], tile_r=2, tile_c=3)
+        close(o2, o, 1e-12)
+        close(lse2, lse, 1e-12)
+
+
+def pin_row_sampling_matches_full(orc):
+    q, k, v = rand(2, 4, 33, 8), rand(2, 2, 33, 8), rand(2, 2, 33, 8)
+    o, lse = orc.attention(q, k, v, 0.35, True, [33, 17], row_block=5)
+    picks = [(0, 0, 0), (1, 3, 32), (1, 1, 16), (0, 2, 20), (1, 2, 20)]
+    o2, lse2 = orc.attention_rows(q, k, v, 0.35, True, [33, 17], picks)
+    for n, (b, h, i) in enumerate(picks):
+        close(o2[n], o[b, h, i], 1e-13)
+        close(lse2[n], lse[b, h, i], 1e-13)
+
+
+def pin_row_block_does_not_change_result(orc):
+    q, k, v = rand(1, 2, 40, 8), rand(1, 1, 40, 8), rand(1, 1, 40, 8)
+    ref = orc.attention(q, k, v, 0.35, True, None, row_block=1024)
+    for rb in (1, 7, 40):
+        got = orc.attention(q, k, v, 0.35, True, None, row_block=rb)
+        close(got[0], ref[0], 1e-13)
+        close(got[1], ref[1], 1e-13)
+
+
+def pin_large_scores_stay_finite(orc):
+    """Scores near ±1000 overflow exp() unless the row max is subtracted first."""
+    q, k, v = rand(1, 1, 8, 4), rand(1, 1, 8, 4), rand(1, 1, 8, 3)
+    o, lse = orc.attention(q, k, v, 0.5, False, None)
+    big = 1000.0 / np.max(np.abs(q))
+    c = 900.0
+    q2 = np.concatenate([q * 1.0, np.full((1, 1, 8, 1), c / 0.5)], axis=3)
+    k2 = np.concatenate([k, np.ones((1, 1, 8, 1))], axis=3)
+    o2, lse2 = orc.attention(q2, k2, v, 0.5, False, None)
+    close(o2, o, 1e-12)
+    close(lse2, lse + c, 1e-12)
+    o3, lse3 = orc.attention(q * big, k, v, 0.5, True, None)
+    assert np.all(np.isfinite(o3)) and np.all(np.isfinite(lse3))
+    for fn in (orc.online_attention_flowchart, orc.online_attention_equations):
+        o4, lse4 = fn(q * big, k, v, 0.5, True, None, tile_r=3, tile_c=2)
+        close(o4, o3, 1e-12)
+        close(lse4, lse3, 1e-12)
+
+
+def _golden_value(x):
+    if isinstance(x, list):
+        return [_golden_value(y) for y in x]
+    if isinstance(x, str):
+        assert x.startswith("ln:")
+        return math.log(float(x[3:]))
+    return x
+
+
+def load_golden(name="hand_worked.json"):
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", name)
+    with open(path, encoding="utf-8") as f:
+        cases = json.load(f)["cases"]
+    out = []
+    for c in cases:
+        out.append({key: (np.array(_golden_value(c[key]), dtype=np.float64)
+                          if key in ("q", "k", "v", "o", "lse") else c[key]) for key in c})
+    return out
+
+
+def pin_hand_worked_golden(orc):
+    """Problems worked by hand (tests/golden/hand_worked.json) to closed-form values."""
+    for c in load_golden():
+        o, lse = orc.attention(c["q"], c["k"], c["v"], c["scale"], c["causal"], c["key_pad_lens"])
+        close(o, c["o"], 1e-14)
+        close(lse, c["lse"], 1e-14)
+
+
+PINS = [f for name, f in sorted(globals().items()) if name.startswith("pin_")]

@@ -1,0 +1,15 @@
+"""B200-native (sm_100a) exact attention forward with the tiled online softmax.
+
+The compute path is the C-ABI library ``libfa.so`` (hand-written CUDA for
+sm_100a, declared in include/fa.h). ``binding`` marshals torch tensors into its
+calls; importing it loads the library and fails loudly when it is missing.
+"""
+
+__all__ = ["fa_fwd", "FaError", "load_library"]
+
+
+def __getattr__(name):
+    if name in __all__:
+        from . import binding
+        return getattr(binding, name)
+    raise AttributeError(name)
