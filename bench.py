@@ -1,0 +1,409 @@
+"""Attention-forward benchmark: TFLOP/s of the sm_100a kernel through the C ABI.
+
+One step = one full forward pass (one fa_fwd launch) over one batch of the
+workload. FLOP = 4·B·Hq·N²·d, halved when causal. Default workload: the GQA
+decoder shape (B=4, Hq=32, Hk=8, N=8192, d=128, bf16, causal), whose inputs
+(402 MB) are larger than L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Multi-GPU (torchrun): every rank runs its own shard of the same workload (a
+different seed: independent batches, no data-path collective; weak scaling);
+timing is the max over ranks. `--impl reference` times the float64 CPU oracle
+on the host cores instead (rank 0 only).
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from tiled_online_softmax_03_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = ("attention fwd TFLOP/s (4·B·Hq·N²·d, ×½ causal) "
+          "and % of B200 BF16 peak")
+FALLBACK_BF16_TFLOPS = 1590.0
+KERNEL_SOURCES = ["tiled_online_softmax_03_b200/csrc/fa_fwd_sm100.cu",
+                  "tiled_online_softmax_03_b200/csrc/fa_ptx.cuh",
+                  "tiled_online_softmax_03_b200/csrc/fa_schedule.cuh"]
+
+
+def flops(w):
+    f = 4.0 * w.B * w.Hq * w.N * w.N * w.d
+    return f * 0.5 if w.causal else f
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return float(m["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, "fallback (1.59 PFLOP/s, earlier measurement on this pool)"
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"fa_fwd_{workload}.md")
+    try:
+        text = open(path, encoding="utf-8").read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_sources_sha256_16") != kernel_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.lines = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                s, m = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            sm.append(s)
+            mx = m
+            for n, flag in zip(names, parts[5:9]):
+                if flag.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = sorted(sm)[len(sm) // 4:] or sm  # drop the idle tail sampled at the edges
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+class OracleSampler:
+    """The float64 oracle, as it stands, timed on bounded samples of the
+    workload: R query rows of one (b, hq) head per call (rows strided across
+    the sequence, heads taken in turn). FLOP are counted as the metric counts
+    them, per row: 4·N·d, halved when causal (a strided row set has the
+    average causal row length)."""
+
+    def __init__(self, w):
+        self.w = w
+        self.x = make_inputs(w)
+        self.G = w.Hq // w.Hk
+        self.heads = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+        self.cache = {}
+        self.calls = 0
+
+    def _head(self, b, h):
+        key = (b, h)
+        if key not in self.cache:
+            self.cache.clear()
+            x, hk = self.x, h // self.G
+            self.cache[key] = (x["q"][b:b + 1, h:h + 1].double().numpy(),
+                               x["k"][b:b + 1, hk:hk + 1].double().numpy(),
+                               x["v"][b:b + 1, hk:hk + 1].double().numpy())
+        return self.cache[key]
+
+    def run(self, rows):
+        """Times one call on `rows` rows; returns (seconds, metric FLOP)."""
+        import oracle
+        w = self.w
+        b, h = self.heads[self.calls % len(self.heads)]
+        stride = max(1, w.N // rows)
+        picks = [(0, 0, (i * stride + self.calls) % w.N) for i in range(rows)]
+        self.calls += 1
+        q, k, v = self._head(b, h)
+        lens = None if self.x["key_pad_lens"] is None else [int(self.x["key_pad_lens"][b])]
+        t0 = time.perf_counter()
+        oracle.attention_rows(q, k, v, w.scale, w.causal, lens, picks)
+        dt = time.perf_counter() - t0
+        per_row = 4.0 * w.N * w.d * (0.5 if w.causal else 1.0)
+        return dt, per_row * rows
+
+
+def oracle_cores():
+    cores = len(os.sched_getaffinity(0))
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 0) for i in threadpool_info()] + [1])
+    except Exception:
+        pass
+    return cores
+
+
+def cpu_baseline(w, budget_s=12.0, rows=256):
+    sampler = OracleSampler(w)
+    sampler.run(8)  # first call pays imports and conversions
+    tot_s, tot_f, calls = 0.0, 0.0, 0
+    while tot_s < budget_s:
+        dt, f = sampler.run(rows)
+        tot_s += dt
+        tot_f += f
+        calls += 1
+    return {"value": tot_f / tot_s / 1e12, "unit": "TFLOP/s", "cores": oracle_cores(),
+            "kind": "oracle",
+            "sample": f"{calls} x {rows} query rows (strided, one (b, hq) head each) of {w.name}, "
+                      f"float64 NumPy oracle, {tot_s:.1f} s of CPU time measured"}
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    sampler = OracleSampler(w)
+    rows = 512
+    for _ in range(args.warmup):
+        sampler.run(rows)
+    tot_s, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, f = sampler.run(rows)
+        tot_s += dt
+        tot_f += f
+    value = tot_f / tot_s / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle_cores(),
+                         "kind": "oracle",
+                         "sample": f"each step {rows} strided query rows of one (b, hq) head of "
+                                   f"{w.name} (float64 oracle)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, n):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hk": w.Hk, "N": w.N, "d": w.d,
+            "causal": w.causal, "key_pad": w.key_pad, "qk_mult": w.qk_mult,
+            "in_dtype": w.dtype, "parallelism": f"independent shards x{n}",
+            "l2": "inputs larger than L2 (no flush)" if in_bytes(w) > 126e6 else
+                  "L2 flushed between steps (256 MB write)"}
+
+
+def in_bytes(w):
+    return 2 * w.B * w.N * w.d * (w.Hq + 2 * w.Hk)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="gqa_8k_causal", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from tiled_online_softmax_03_b200 import binding
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    x = make_inputs(w, batch_offset=rank)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    lens = x["key_pad_lens"].to(dev) if x["key_pad_lens"] is not None else None
+    o = torch.empty_like(q)
+    lse = torch.empty(w.B, w.Hq, w.N, dtype=torch.float32, device=dev)
+    flush = None
+    if in_bytes(w) <= 126e6:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        if flush is not None:
+            flush.fill_(1)
+        binding.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, key_pad_lens=lens, out=o, lse=lse,
+                       stream=stream.cuda_stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+
+    # ---- device-timed loop: events around every launch, on the launching stream
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        t_begin.record(stream)
+        for i in range(args.steps):
+            if flush is not None:
+                flush.fill_(1)
+            starts[i].record(stream)
+            binding.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, key_pad_lens=lens, out=o,
+                           lse=lse, stream=stream.cuda_stream)
+            ends[i].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    status = binding.device_status()
+    total_ms = max_over_ranks(t_begin.elapsed_time(t_end))
+    kern_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    kern_avg = max_over_ranks(sum(kern_ms) / len(kern_ms))
+
+    # ---- end-to-end through the public API: pinned host inputs in, O and LSE out
+    hq_, hk_, hv_ = (x[n].pin_memory() for n in ("q", "k", "v"))
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    hlens = x["key_pad_lens"].pin_memory() if x["key_pad_lens"] is not None else None
+    e2e_steps = max(1, min(args.e2e_steps, args.steps))
+
+    def e2e_step():
+        q.copy_(hq_, non_blocking=True)
+        k.copy_(hk_, non_blocking=True)
+        v.copy_(hv_, non_blocking=True)
+        if hlens is not None:
+            lens.copy_(hlens, non_blocking=True)
+        binding.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, key_pad_lens=lens, out=o, lse=lse,
+                       stream=stream.cuda_stream)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+    h2d = sum(t.numel() * t.element_size() for t in (hq_, hk_, hv_)) + \
+        (hlens.numel() * 4 if hlens is not None else 0)
+    d2h = ho.numel() * ho.element_size() + hl.numel() * 4
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    f = flops(w)
+    ms_per_step = total_ms / args.steps
+    value = f * world / (ms_per_step * 1e-3) / 1e12
+    peak, peak_src = peaks()
+    achieved = f / (kern_avg * 1e-3) / 1e12
+    traffic = recorded_traffic(w.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
+        "config": config_of(w, world),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                     "kernel": "fa_fwd_kernel", "kernel_ms": kern_avg,
+                     "flop_per_launch": f},
+        "e2e": {"value": f * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+        "device_status": status,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = {k2: v2 for k2, v2 in cpu_baseline(w).items()
+                                if k2 not in ("seconds", "heads")}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

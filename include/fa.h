@@ -1,0 +1,130 @@
+/*
+ * fa.h — C ABI of libfa.so: exact attention forward on B200 (sm_100a).
+ *
+ * The operation (page "FlashAttention (VI)", section "Vấn đề của cơ chế
+ * attention tiêu chuẩn", plus the masks of "FlashAttention 在昇腾 NPU 上是怎么
+ * 省显存的？…" sections "坑一" (causal) and "坑四" (GQA/MQA)):
+ *
+ *     S   = scale · Q Kᵀ + mask          (mask: 0 or −inf)
+ *     O   = softmax_rows(S) · V
+ *     LSE = ln Σ_j exp(S_ij)             (per query row, natural log)
+ *
+ * computed tile by tile with the online-softmax recurrence of "MCU 上
+ * Transformer 模型的 Flash Attention 实现在 256KB SRAM 约束下的分块计算与内存
+ * 建模方案", §二 (running row max m, running denominator l, rescaled O,
+ * division by l at the end), so the N×N matrix S never reaches memory.
+ *
+ * Masks. Key j is allowed for query row i when j < L_b (key padding; L_b =
+ * key_pad_lens[b] clamped to [0, N], or N when key_pad_lens is NULL) and,
+ * with causal != 0, when j <= i. Every query row is computed, including rows
+ * i >= L_b. A row with no allowed key gets O = 0 and LSE = −inf.
+ *
+ * GQA/MQA. Query head hq reads K/V head hq / (Hq / Hk) (contiguous groups).
+ *
+ * Layouts (all contiguous, row-major, same 16-bit dtype for q, k, v, o):
+ *     q, o : [B, Hq, N, d]        k, v : [B, Hk, N, d]
+ *     lse  : [B, Hq, N] float32   key_pad_lens : [B] int32
+ *
+ * Ownership. The caller allocates every buffer (device memory) and owns the
+ * stream. The library allocates nothing per call and keeps no pointer after
+ * the call returns. o and lse must not overlap q, k, v or each other.
+ *
+ * Asynchrony and errors. fa_fwd validates its arguments on the host and
+ * returns a negative fa_status without launching anything when they are
+ * invalid; otherwise it enqueues one kernel on `stream` and returns FA_OK
+ * (or FA_ERR_CUDA if the launch itself failed). The kernel never traps: each
+ * of its waits is bounded, and a wait that runs out records
+ * FA_ERR_DEVICE_TIMEOUT in a per-device status word that
+ * fa_get_device_status() reads. Messages for the last host-side error of the
+ * calling thread come from fa_last_error_string().
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_FP16 = 0, /* IEEE binary16 inputs and output */
+  FA_BF16 = 1  /* bfloat16 inputs and output */
+} fa_dtype;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = -1,    /* NULL pointer, bad size, misaligned buffer, non-finite scale */
+  FA_ERR_UNSUPPORTED = -2,    /* head dim other than 64 or 128, unknown dtype */
+  FA_ERR_CUDA = -3,           /* a CUDA runtime/driver call or the launch failed */
+  FA_ERR_DEVICE_TIMEOUT = -4  /* a bounded wait inside the kernel ran out */
+} fa_status;
+
+/*
+ * fa_fwd — one attention forward pass (the whole hot path, one launch).
+ *
+ *   q, k, v      device pointers, 16-byte aligned, dtype `dtype`.
+ *   o            device pointer [B, Hq, N, d], written.
+ *   lse          device pointer [B, Hq, N] float32, written; NULL skips it.
+ *   B, Hq, Hk, N batch, query heads, K/V heads, sequence length; all >= 1,
+ *                Hq % Hk == 0.
+ *   d            head dimension: 64 or 128 (the pages ask for a multiple of
+ *                16 and use 64 and 128; other values return
+ *                FA_ERR_UNSUPPORTED instead of falling back silently).
+ *   scale        finite multiplier of Q Kᵀ (usually 1/sqrt(d)); any sign.
+ *   causal       0 or 1.
+ *   key_pad_lens device pointer to B int32 valid-key counts, or NULL.
+ *                Values are clamped to [0, N] in the kernel.
+ *   stream       a cudaStream_t (NULL = legacy default stream).
+ *   dtype        FA_FP16 or FA_BF16.
+ * Returns FA_OK or a negative fa_status.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int Hq, int Hk, int N, int d, float scale, int causal,
+           const int32_t* key_pad_lens, void* stream, int dtype);
+
+/* Message for the last error returned to the calling thread ("" if none).
+ * The string is owned by the library (thread-local storage). */
+const char* fa_last_error_string(void);
+
+/* Synchronises the current device, then returns and clears its status word:
+ * FA_OK, FA_ERR_DEVICE_TIMEOUT, or FA_ERR_CUDA if reading it failed. */
+int fa_get_device_status(void);
+
+/* Bound on each in-kernel wait, in milliseconds (default 4000; 1..600000).
+ * Returns FA_OK or FA_ERR_INVALID_ARG. Applies to later launches. */
+int fa_set_wait_timeout_ms(int ms);
+
+/* ---- schedule introspection (host only; no GPU needed) ------------------
+ * The kernel splits the query side into work units of two 128-row Q tiles
+ * that share one K/V head: the tiles of one (b, hk) are enumerated by
+ * (m-block, query head in the group) and paired in that order. Causal
+ * problems list units heaviest first (largest m-block first); each CTA of a
+ * persistent grid takes units in a serpentine order. */
+
+/* Number of work units for a problem shape; < 0 on bad arguments. */
+int fa_num_units(int B, int Hq, int Hk, int N, int causal);
+
+/* Decodes unit u into out[8] = {b, hk, hq0, mblock0, present0, hq1, mblock1,
+ * present1}. Returns FA_OK or FA_ERR_INVALID_ARG. */
+int fa_unit_info(int B, int Hq, int Hk, int N, int causal, int u, int32_t* out);
+
+/* Unit taken by CTA `cta` of a `grid`-CTA launch on its iteration `it`
+ * (may be >= fa_num_units, meaning that CTA is done). */
+int fa_unit_for(int cta, int it, int grid);
+
+/* Self test of the bounded wait: launches one thread that waits on an
+ * mbarrier nothing arrives at, with a limit of `ms` (1..10000) milliseconds,
+ * on the legacy default stream, and synchronises. Returns FA_OK when the wait
+ * gave up as designed (FA_ERR_DEVICE_TIMEOUT is then left in the status word),
+ * FA_ERR_CUDA otherwise. Allocates 8 bytes of device memory for the result. */
+int fa_selftest_wait_timeout(int ms);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

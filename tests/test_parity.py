@@ -1,0 +1,166 @@
+"""CUDA path (through the C ABI) against the float64 oracle, element by element.
+
+Small problems are compared on every output; the full-size workloads are
+compared on sampled rows that the oracle computes one by one, in the same
+launch configuration the benchmark times.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import (compare, oracle_full, oracle_rows, run_cuda, sample_picks, to64)
+from tiled_online_softmax_03_b200.inputs import WORKLOADS, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _need_cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def small(B, Hq, Hk, N, d, dtype, causal, lens=None, seed=0, qk_mult=1.0):
+    w = Workload("t", B, Hq, Hk, N, d, dtype, causal, qk_mult=qk_mult, seed=seed)
+    x = make_inputs(w)
+    if lens is not None:
+        x["key_pad_lens"] = torch.tensor(lens, dtype=torch.int32)
+    return w, x
+
+
+def check_full(w, x, scale=None):
+    scale = w.scale if scale is None else scale
+    o, lse = run_cuda(x["q"], x["k"], x["v"], w.causal, scale, x["key_pad_lens"])
+    o_ref, lse_ref = oracle_full(x["q"], x["k"], x["v"], w.causal, scale, x["key_pad_lens"])
+    return compare(to64(o), to64(lse), o_ref, lse_ref, w.torch_dtype)
+
+
+# ------------------------------------------------------------- small shapes
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 17, 127, 128, 129, 300, 513])
+def test_ragged_lengths(N, causal, d, dtype):
+    w, x = small(1, 2, 1, N, d, dtype, causal, seed=N + 7 * d)
+    check_full(w, x)
+
+
+@pytest.mark.parametrize("Hq,Hk", [(1, 1), (2, 2), (4, 2), (8, 2), (6, 2), (3, 1), (32, 1), (8, 8)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_head_groups(Hq, Hk, causal):
+    w, x = small(2, Hq, Hk, 384, 128, "bf16", causal, seed=Hq * 10 + Hk)
+    check_full(w, x)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_key_padding_edges(causal, d):
+    # lengths 0 (every row empty), 1, a tile edge, ragged, and N itself
+    lens = [0, 1, 128, 200, 384, 383]
+    w, x = small(len(lens), 4, 2, 384, d, "bf16", causal, lens=lens, seed=3 + d)
+    check_full(w, x)
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.2, 0.5])
+def test_scale_values(scale):
+    w, x = small(1, 2, 2, 300, 64, "fp16", True, seed=11)
+    check_full(w, x, scale=scale)
+
+
+def test_peaked_rows_stress_rescale():
+    # Q, K scaled by 3 (the long-context recipe) at a size the oracle finishes quickly
+    w, x = small(1, 4, 2, 1024, 128, "bf16", True, seed=5, qk_mult=3.0)
+    check_full(w, x)
+
+
+def test_increasing_scores_force_every_rescale():
+    # scores grow along the key axis, so the running max moves on every K/V tile
+    w, x = small(1, 1, 1, 1024, 64, "bf16", False, seed=9)
+    ramp = torch.linspace(-30, 30, 1024).reshape(1, 1, 1024, 1)
+    x["k"] = (torch.zeros(1, 1, 1024, 64) + ramp / 8).to(torch.bfloat16)
+    x["q"] = torch.ones(1, 1, 1024, 64, dtype=torch.bfloat16)
+    check_full(w, x)
+
+
+# ------------------------------------------------------- the five workloads
+
+def test_single_head_128_full():
+    w = WORKLOADS["single_head_128"]
+    check_full(w, make_inputs(w))
+
+
+def test_bert_large_512_keypad_full():
+    w = WORKLOADS["bert_large_512_keypad"]
+    check_full(w, make_inputs(w))
+
+
+@pytest.mark.parametrize("name", ["llama7b_4k_causal", "gqa_8k_causal", "mqa_8k_causal",
+                                  "long_32k_causal"])
+def test_full_size_sampled_rows(name):
+    w = WORKLOADS[name]
+    x = make_inputs(w)
+    o, lse = run_cuda(x["q"], x["k"], x["v"], w.causal, w.scale, x["key_pad_lens"])
+    picks = sample_picks(w.B, w.Hq, w.N, 160, seed=w.seed)
+    o_ref, lse_ref = oracle_rows(x["q"], x["k"], x["v"], w.causal, w.scale, x["key_pad_lens"],
+                                 picks)
+    idx = tuple(np.array(picks).T)
+    o_s = to64(o)[idx]
+    lse_s = to64(lse)[idx]
+    compare(o_s, lse_s, o_ref, lse_ref, w.torch_dtype)
+    # properties that hold at any size: finite everywhere, causal row 0 is V row 0
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    G = w.Hq // w.Hk
+    v0 = x["v"][:, torch.arange(w.Hq) // G, 0].to(o.device)
+    assert torch.equal(o[:, :, 0], v0)
+
+
+def test_llama7b_4k_two_heads_full():
+    w = WORKLOADS["llama7b_4k_causal"]
+    x = make_inputs(w)
+    o, lse = run_cuda(x["q"], x["k"], x["v"], w.causal, w.scale, None)
+    for h in (0, w.Hq - 1):
+        o_ref, lse_ref = oracle_full(x["q"][:, h:h + 1], x["k"][:, h:h + 1], x["v"][:, h:h + 1],
+                                     True, w.scale, None)
+        compare(to64(o[:, h:h + 1]), to64(lse[:, h:h + 1]), o_ref, lse_ref, w.torch_dtype)
+
+
+# -------------------------------------------------------------- exact cases
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_causal_row0_is_exact(dtype):
+    w, x = small(2, 4, 2, 777, 128, dtype, True, seed=21)
+    o, lse = run_cuda(x["q"], x["k"], x["v"], True, w.scale, None)
+    G = 2
+    v0 = x["v"][:, torch.arange(4) // G, 0].to(o.device)
+    assert torch.equal(o[:, :, 0], v0)
+    s00 = w.scale * (to64(x["q"][:, :, 0]) * to64(x["k"][:, torch.arange(4) // G, 0])).sum(-1)
+    assert np.max(np.abs(to64(lse[:, :, 0]) - s00)) < 1e-4
+
+
+def test_single_key_rows_are_exact():
+    lens = [1, 1]
+    w, x = small(2, 2, 1, 256, 64, "bf16", False, lens=lens, seed=4)
+    o, _ = run_cuda(x["q"], x["k"], x["v"], False, w.scale, x["key_pad_lens"])
+    want = x["v"][:, [0, 0], 0:1].expand(2, 2, 256, 64).to(o.device)
+    assert torch.equal(o, want)
+
+
+def test_uniform_v_is_reproduced():
+    w, x = small(1, 2, 2, 640, 128, "bf16", True, seed=8)
+    row = torch.randn(128).to(torch.bfloat16)
+    x["v"] = row.expand(1, 2, 640, 128).contiguous()
+    o, _ = run_cuda(x["q"], x["k"], x["v"], True, w.scale, None)
+    err = (o.float().cpu() - row.float()).abs().max().item()
+    ulp = row.float().abs().max().item() * 2 ** -7
+    assert err <= ulp
+
+
+def test_deterministic_and_stream():
+    w, x = small(2, 8, 2, 1000, 128, "bf16", True, seed=1)
+    o1, l1 = run_cuda(x["q"], x["k"], x["v"], True, w.scale, None)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o2, l2 = run_cuda(x["q"], x["k"], x["v"], True, w.scale, None,
+                          stream=s.cuda_stream)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)

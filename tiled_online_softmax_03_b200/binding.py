@@ -1,0 +1,134 @@
+"""ctypes binding of libfa.so (include/fa.h): argument marshalling only.
+
+Every step of the attention forward runs in the library's CUDA kernel; this
+module checks tensor metadata, allocates the outputs with torch when the
+caller does not pass them, and calls ``fa_fwd`` on the current torch stream.
+Importing it loads the library and raises if it is missing: there is no
+fallback path.
+"""
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["FaError", "fa_fwd", "load_library", "lib", "FA_OK", "FA_ERR_INVALID_ARG",
+           "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT"]
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = -1
+FA_ERR_UNSUPPORTED = -2
+FA_ERR_CUDA = -3
+FA_ERR_DEVICE_TIMEOUT = -4
+FA_FP16 = 0
+FA_BF16 = 1
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
+
+
+class FaError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"fa error {code}: {msg}")
+        self.code = code
+
+
+def load_library(path=LIB_PATH):
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build it with `python -m tiled_online_softmax_03_b200.build` "
+            "(there is no non-CUDA fallback)")
+    L = ctypes.CDLL(path)
+    c_int, c_void_p, c_float = ctypes.c_int, ctypes.c_void_p, ctypes.c_float
+    L.fa_fwd.argtypes = [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
+                         c_int, c_int, c_float, c_int, c_void_p, c_void_p, c_int]
+    L.fa_fwd.restype = c_int
+    L.fa_last_error_string.argtypes = []
+    L.fa_last_error_string.restype = ctypes.c_char_p
+    L.fa_get_device_status.argtypes = []
+    L.fa_get_device_status.restype = c_int
+    L.fa_set_wait_timeout_ms.argtypes = [c_int]
+    L.fa_set_wait_timeout_ms.restype = c_int
+    L.fa_num_units.argtypes = [c_int] * 5
+    L.fa_num_units.restype = c_int
+    L.fa_unit_info.argtypes = [c_int] * 6 + [ctypes.POINTER(ctypes.c_int32)]
+    L.fa_unit_info.restype = c_int
+    L.fa_unit_for.argtypes = [c_int] * 3
+    L.fa_unit_for.restype = c_int
+    L.fa_selftest_wait_timeout.argtypes = [c_int]
+    L.fa_selftest_wait_timeout.restype = c_int
+    L.fa_version.argtypes = []
+    L.fa_version.restype = c_int
+    return L
+
+
+lib = load_library()
+
+
+def last_error():
+    return lib.fa_last_error_string().decode(errors="replace")
+
+
+def check(code):
+    if code != FA_OK:
+        raise FaError(code, last_error())
+    return code
+
+
+_DTYPES = {torch.float16: FA_FP16, torch.bfloat16: FA_BF16}
+
+
+def fa_fwd(q, k, v, causal=False, scale=None, key_pad_lens=None, out=None, lse=None,
+           return_lse=True, stream=None):
+    """O (and LSE) = attention forward of q [B,Hq,N,d] against k, v [B,Hk,N,d].
+
+    Tensors must be CUDA, contiguous, fp16 or bf16 (all the same). ``scale``
+    defaults to 1/sqrt(d). ``key_pad_lens`` is an int32 CUDA tensor [B] or
+    None. ``out``/``lse`` may be given preallocated. Returns (o, lse) or o.
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise FaError(FA_ERR_INVALID_ARG, f"{name} must be a contiguous 4-D CUDA tensor")
+    if q.dtype not in _DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise FaError(FA_ERR_UNSUPPORTED, "q, k, v must share one dtype: float16 or bfloat16")
+    B, Hq, N, d = q.shape
+    Hk = k.shape[1]
+    if tuple(k.shape) != (B, Hk, N, d) or tuple(v.shape) != (B, Hk, N, d):
+        raise FaError(FA_ERR_INVALID_ARG, "k and v must be [B, Hk, N, d] matching q")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    if key_pad_lens is not None:
+        if key_pad_lens.dtype != torch.int32 or not key_pad_lens.is_cuda or \
+                key_pad_lens.numel() != B:
+            raise FaError(FA_ERR_INVALID_ARG, "key_pad_lens must be an int32 CUDA tensor [B]")
+    if scale is None:
+        scale = float(d) ** -0.5
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    with torch.cuda.device(q.device):
+        check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                         lse.data_ptr() if lse is not None else None, B, Hq, Hk, N, d,
+                         float(scale), 1 if causal else 0,
+                         key_pad_lens.data_ptr() if key_pad_lens is not None else None,
+                         stream, _DTYPES[q.dtype]))
+    return (out, lse) if return_lse else out
+
+
+def device_status():
+    """Synchronise and read (then clear) the kernel's device status word."""
+    return lib.fa_get_device_status()
+
+
+def num_units(B, Hq, Hk, N, causal):
+    return lib.fa_num_units(B, Hq, Hk, N, 1 if causal else 0)
+
+
+def unit_info(B, Hq, Hk, N, causal, u):
+    out = (ctypes.c_int32 * 8)()
+    check(lib.fa_unit_info(B, Hq, Hk, N, 1 if causal else 0, u, out))
+    return list(out)
+
+
+def unit_for(cta, it, grid):
+    return lib.fa_unit_for(cta, it, grid)

@@ -1,0 +1,965 @@
+// fa_fwd_sm100.cu — exact attention forward for B200 (sm_100a) and its C ABI.
+//
+// What it computes: O = softmax(scale·QKᵀ + mask)·V and LSE per query row
+// (page "FlashAttention (VI)", section "Vấn đề của cơ chế attention tiêu
+// chuẩn"), tile by tile with the online-softmax recurrence of the page "MCU 上
+// Transformer 模型的 Flash Attention 实现在 256KB SRAM 约束下的分块计算与内存建模
+// 方案", §二: per query row a running max m, a running denominator l and an
+// unnormalised O, rescaled by exp(m_old − m_new) when m grows, divided by l once
+// at the end (§三). Scores never leave the SM: S lives in tensor memory (TMEM),
+// P overwrites it there, only O and LSE are written to HBM.
+//
+// One persistent CTA per SM (512 threads, one 512-column TMEM allocation)
+// walks work units of two 128-row Q tiles that share a K/V head
+// (fa_schedule.cuh). Warp roles:
+//   warps 0-3   softmax for Q tile 0 (thread r owns row r: TMEM lane r)
+//   warps 4-7   softmax for Q tile 1
+//   warps 8-11  correction (rescale O in TMEM) and epilogue (O/l, LSE, stores)
+//   warp 12     tcgen05.mma issue (one thread)
+//   warp 13     TMA loads (one thread)
+//   warps 14-15 no work
+// Per K/V tile j and Q tile t the MMA thread issues S_t = Q_t·K_jᵀ into TMEM,
+// the softmax warps turn S_t into P_t (16-bit, written over S_t in TMEM) and
+// the running statistics, the correction warps rescale O_t, and the MMA thread
+// issues O_t += P_t·V_j with P read from TMEM. The two Q tiles alternate, so
+// the tensor core works on one tile while the other tile's softmax runs.
+//
+// Pipelines use mbarriers; every wait is bounded (globaltimer) and a wait that
+// runs out records FA_ERR_DEVICE_TIMEOUT in g_fa_status instead of hanging.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "fa_ptx.cuh"
+#include "fa_schedule.cuh"
+
+namespace fa {
+
+__device__ int g_fa_status;  // first device-side error of any launch (0 = none)
+
+constexpr int NUM_THREADS = 512;
+constexpr int TMEM_COLS = 512;
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: keep a stale max until it is 2^8 behind
+constexpr int SW128_BOX_BYTES = BM * 128;  // one 128-row box of 64 16-bit columns
+constexpr int OST_BYTES = 32 * 32 * 2;     // one 32-row × 32-column output staging box
+
+// TMEM columns: S/P for tile 0 and 1, then O for tile 0 and 1.
+__device__ constexpr uint32_t S_COL[2] = {0, 128};
+template <int D>
+struct TmemO {
+  __host__ __device__ static constexpr uint32_t col(int t) { return 256 + t * D; }
+};
+
+// Barrier slots.
+enum {
+  BAR_QFULL = 0,    // [2] TMA -> MMA: Q tile loaded
+  BAR_QEMPTY = 2,   // [2] MMA -> TMA: all QK of the unit done with Q tile
+  BAR_SFULL = 4,    // [2] MMA -> softmax: S tile ready in TMEM
+  BAR_PFULL = 6,    // [2] softmax -> MMA: P written to TMEM
+  BAR_AFULL = 8,    // [2] softmax -> correction: rescale factors in smem
+  BAR_OCORR = 10,   // [2] correction -> MMA: O rescaled
+  BAR_PVDONE = 12,  // [2] MMA -> epilogue: last P·V of the unit done
+  BAR_OFREE = 14,   // [2] epilogue -> MMA: O read out of TMEM
+  BAR_STATS = 16,   // [2 tiles][2 buffers] softmax -> epilogue: final m, l in smem
+  BAR_DRAIN = 20,   // MMA drain on the abort path
+  BAR_KV = 21       // [STAGES] full, then [STAGES] empty
+};
+
+template <int D>
+struct Layout {
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int STAGES = (D == 128) ? 4 : 8;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_OST = OFF_KV + STAGES * KV_BYTES;
+  static constexpr int OFF_ALPHA = OFF_OST + 8 * OST_BYTES;   // [2 tiles][128] float
+  static constexpr int OFF_STATS = OFF_ALPHA + 2 * BM * 4;    // [2 buf][2 tiles][128] float4
+  static constexpr int OFF_BAR = OFF_STATS + 2 * 2 * BM * 16;
+  static constexpr int NUM_BARS = BAR_KV + 2 * STAGES;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;     // tmem base, abort flag
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;                  // base is rounded up to 1 KB
+  static_assert(OFF_KV % 1024 == 0 && OFF_OST % 2048 == 0, "tile alignment");
+  static_assert(ALLOC <= 232448, "shared memory budget");
+};
+
+struct Params {
+  const int32_t* key_pad_lens;
+  float* lse;
+  Shape s;
+  float scale_log2;
+  unsigned long long timeout_ns;
+};
+
+// ------------------------------------------------------------ descriptors
+// UMMA shared-memory descriptor, sm_100 format: start address >> 4 in bits
+// 0-13, leading byte offset >> 4 in 16-29, stride byte offset >> 4 in 32-45,
+// version 1 in bit 46, layout (2 = 128-byte swizzle) in bits 61-63.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr & 0x3FFFF) >> 4) | ((uint64_t)(lbo >> 4) << 16) |
+         ((uint64_t)(sbo >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor for kind::f16 with fp32 accumulation, M = 128.
+__host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int n, bool b_mn_major) {
+  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
+         ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+// ------------------------------------------------------------ bounded waits
+struct Ctl {
+  volatile int* abort_flag;
+  unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, const Ctl& c) {
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*c.abort_flag) return false;
+    if (global_timer_ns() - t0 > c.timeout_ns) {
+      *c.abort_flag = 1;
+      atomicCAS(&g_fa_status, 0, (int)FA_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& c) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_slow(bar, parity, c);
+}
+// Warp-uniform form for roles whose later instructions are warp-collective.
+__device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, const Ctl& c) {
+  const bool ok = wait_bar(bar, parity, c);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int D>
+__device__ __forceinline__ uint32_t bar_addr(uint32_t sbase, int i) {
+  return sbase + Layout<D>::OFF_BAR + 8 * i;
+}
+
+__device__ __forceinline__ int key_len_of(const Params& p, int b) {
+  if (p.key_pad_lens == nullptr) return p.s.N;
+  int l = __ldg(p.key_pad_lens + b);
+  return l < 0 ? 0 : (l > p.s.N ? p.s.N : l);
+}
+
+__device__ __forceinline__ bool next_unit(const Params& p, int it, Unit& U) {
+  const int u = unit_for(blockIdx.x, it, gridDim.x);
+  if (u >= p.s.num_units) return false;
+  decode_unit(p.s, u, U);
+  resolve_unit(p.s, key_len_of(p, U.b), U);
+  return true;
+}
+
+// ============================================================ TMA producer
+template <int D>
+__device__ void role_load(const Params& p, uint32_t sbase, const Ctl& c, const CUtensorMap* tm_q,
+                          const CUtensorMap* tm_k, const CUtensorMap* tm_v) {
+  using L = Layout<D>;
+  uint32_t qe_ph[2] = {0, 0};
+  int st = 0;
+  uint32_t kv_ph = 0;
+  // parity of the last arming of each barrier, for the abort drain
+  uint32_t armed_q = 0, armed_kv = 0, last_q_ph[2] = {0, 0}, last_kv_ph[L::STAGES];
+  bool ok = true;
+  Unit U;
+  for (int it = 0; ok && next_unit(p, it, U); ++it) {
+    for (int t = 0; t < 2 && ok; ++t) {
+      if (U.n[t] == 0) continue;
+      if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_QEMPTY + t), qe_ph[t] ^ 1, c))) break;
+      qe_ph[t] ^= 1;
+      const uint32_t full = bar_addr<D>(sbase, BAR_QFULL + t);
+      mbar_arrive_expect_tx(full, L::Q_BYTES);
+      last_q_ph[t] = (armed_q >> t & 1) ? last_q_ph[t] ^ 1 : 0;
+      armed_q |= 1u << t;
+      const int head = U.b * p.s.Hq + U.hq[t];
+      for (int bx = 0; bx < D / 64; ++bx)
+        tma_load_3d(sbase + L::OFF_Q + t * L::Q_BYTES + bx * SW128_BOX_BYTES, tm_q, bx * 64,
+                    U.mb[t] * BM, head, full);
+    }
+    const int kv_head = U.b * p.s.Hk + U.hk;
+    for (int j = 0; j < U.nmax && ok; ++j) {
+      for (int which = 0; which < 2; ++which) {  // K_j then V_j
+        if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_KV + L::STAGES + st), kv_ph ^ 1, c))) break;
+        const uint32_t full = bar_addr<D>(sbase, BAR_KV + st);
+        mbar_arrive_expect_tx(full, L::KV_BYTES);
+        last_kv_ph[st] = kv_ph;
+        armed_kv |= 1u << st;
+        const CUtensorMap* map = which ? tm_v : tm_k;
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_load_3d(sbase + L::OFF_KV + st * L::KV_BYTES + bx * SW128_BOX_BYTES, map, bx * 64,
+                      j * BN, kv_head, full);
+        if (++st == L::STAGES) {
+          st = 0;
+          kv_ph ^= 1;
+        }
+      }
+    }
+  }
+  if (!ok) {
+    // Let every armed copy land before the CTA can exit (bounded, short).
+    Ctl drain{c.abort_flag, 100000000ull};
+    volatile int no_abort = 0;
+    drain.abort_flag = &no_abort;
+    for (int t = 0; t < 2; ++t)
+      if (armed_q >> t & 1) wait_bar(bar_addr<D>(sbase, BAR_QFULL + t), last_q_ph[t], drain);
+    for (int s = 0; s < L::STAGES; ++s)
+      if (armed_kv >> s & 1) wait_bar(bar_addr<D>(sbase, BAR_KV + s), last_kv_ph[s], drain);
+  }
+}
+
+// ============================================================= MMA issuer
+template <int D, bool BF16>
+__device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const Ctl& c) {
+  using L = Layout<D>;
+  constexpr uint32_t IDESC_QK = idesc_f16(BF16, BN, false);  // S = Q·Kᵀ, both K-major
+  constexpr uint32_t IDESC_PV = idesc_f16(BF16, D, true);    // O += P·V, V is MN-major
+  uint32_t qf_ph[2] = {0, 0}, pf_ph[2] = {0, 0}, oc_ph[2] = {0, 0}, of_ph[2] = {0, 0};
+  int st = 0;
+  uint32_t kv_ph = 0;
+  bool ok = true;
+
+  // Descriptors are built once per operand tile; a K step adds its byte
+  // offset >> 4 to the start-address field (bits 0-13, no carry out: < 256 KB).
+  auto issue_qk = [&](int t, int kst) {
+    const uint64_t qd = sdesc(sbase + L::OFF_Q + t * L::Q_BYTES, 16, 1024);
+    const uint64_t kd = sdesc(sbase + L::OFF_KV + kst * L::KV_BYTES, 16, 1024);
+    const uint32_t d_s = tmem + S_COL[t];
+#pragma unroll 1
+    for (int k = 0; k < D / 16; ++k) {
+      const uint32_t off = ((k >> 2) * SW128_BOX_BYTES + (k & 3) * 32) >> 4;
+      umma_ss(d_s, qd + off, kd + off, IDESC_QK, k > 0);
+    }
+  };
+  auto issue_pv = [&](int t, int vst, bool acc) {
+    // P: 16 keys = 8 TMEM columns (two 16-bit values per column); V: 16 key
+    // rows of 128 bytes in each 64-column box, boxes SW128_BOX_BYTES apart.
+    const uint64_t vd = sdesc(sbase + L::OFF_KV + vst * L::KV_BYTES, SW128_BOX_BYTES, 1024);
+    const uint32_t d_o = tmem + TmemO<D>::col(t);
+    const uint32_t a_p = tmem + S_COL[t];
+#pragma unroll 1
+    for (int k = 0; k < BN / 16; ++k)
+      umma_ts(d_o, a_p + k * 8, vd + ((k * 16 * 128) >> 4), IDESC_PV, (acc || k > 0) ? 1u : 0u);
+  };
+
+  Unit U;
+  for (int it = 0; ok && next_unit(p, it, U); ++it) {
+    if (U.nmax == 0) continue;
+    const int k0 = st;
+    const uint32_t k0_ph = kv_ph;
+    if (++st == L::STAGES) { st = 0; kv_ph ^= 1; }
+    if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_KV + k0), k0_ph, c))) break;
+    for (int t = 0; t < 2 && ok; ++t) {
+      if (U.n[t] == 0) continue;
+      if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_QFULL + t), qf_ph[t], c))) break;
+      qf_ph[t] ^= 1;
+    }
+    if (!ok) break;
+    tc_fence_after();
+    for (int t = 0; t < 2; ++t) {
+      if (U.n[t] == 0) continue;
+      issue_qk(t, k0);
+      umma_commit(bar_addr<D>(sbase, BAR_SFULL + t));
+    }
+    umma_commit(bar_addr<D>(sbase, BAR_KV + L::STAGES + k0));
+
+    for (int j = 0; j < U.nmax && ok; ++j) {
+      const int vs = st;
+      const uint32_t vs_ph = kv_ph;
+      if (++st == L::STAGES) { st = 0; kv_ph ^= 1; }
+      int kn = -1;
+      uint32_t kn_ph = 0;
+      if (j + 1 < U.nmax) {
+        kn = st;
+        kn_ph = kv_ph;
+        if (++st == L::STAGES) { st = 0; kv_ph ^= 1; }
+      }
+      if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_KV + vs), vs_ph, c))) break;
+      bool kn_ready = false;
+      for (int t = 0; t < 2; ++t) {
+        if (j >= U.n[t]) continue;
+        if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_PFULL + t), pf_ph[t], c))) break;
+        pf_ph[t] ^= 1;
+        if (j > 0) {
+          if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_OCORR + t), oc_ph[t], c))) break;
+          oc_ph[t] ^= 1;
+        } else {
+          if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_OFREE + t), of_ph[t] ^ 1, c))) break;
+          of_ph[t] ^= 1;
+        }
+        tc_fence_after();
+        issue_pv(t, vs, j > 0);
+        if (j == U.n[t] - 1) {
+          umma_commit(bar_addr<D>(sbase, BAR_PVDONE + t));
+          umma_commit(bar_addr<D>(sbase, BAR_QEMPTY + t));
+        } else {
+          if (!kn_ready) {
+            if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_KV + kn), kn_ph, c))) break;
+            kn_ready = true;
+            tc_fence_after();
+          }
+          issue_qk(t, kn);
+          umma_commit(bar_addr<D>(sbase, BAR_SFULL + t));
+        }
+      }
+      if (!ok) break;
+      umma_commit(bar_addr<D>(sbase, BAR_KV + L::STAGES + vs));
+      if (kn >= 0) umma_commit(bar_addr<D>(sbase, BAR_KV + L::STAGES + kn));
+    }
+  }
+  if (!ok) {
+    // Let every issued MMA finish before TMEM is released.
+    volatile int no_abort = 0;
+    Ctl drain{&no_abort, 100000000ull};
+    umma_commit(bar_addr<D>(sbase, BAR_DRAIN));
+    wait_bar(bar_addr<D>(sbase, BAR_DRAIN), 0, drain);
+  }
+}
+
+// ================================================================= softmax
+// Rounds (lo, hi) to the 16-bit MMA type and packs them as one TMEM column
+// (lo in the low half). `sum_r` accumulates the rounded values (what the P·V
+// product consumes), `sum_e` the unrounded ones.
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi, float& sum_r, float& sum_e) {
+  sum_e += lo + hi;
+  if constexpr (BF16) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    const float2 f = __bfloat1622float2(h);
+    sum_r += f.x + f.y;
+    return *reinterpret_cast<uint32_t*>(&h);
+  } else {
+    __half2 h = __floats2half2_rn(lo, hi);
+    const float2 f = __half22float2(h);
+    sum_r += f.x + f.y;
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+// Row max of one S tile for this thread's row, in log2 units of the scaled
+// score. MASKED: keys c >= nvalid are masked, and s is rewritten in place to
+// s·scale·log2e (−inf where masked); otherwise s stays raw and the max of the
+// scaled row is taken as max(s)·k for k >= 0, min(s)·k for k < 0.
+template <bool MASKED>
+__device__ __forceinline__ float row_max(uint32_t (&s)[BN], float sl2, int nvalid) {
+  float mx[8];
+  if constexpr (!MASKED) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(s[i]);
+    if (sl2 >= 0.f) {
+#pragma unroll
+      for (int i = 8; i < BN; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(s[i]));
+      return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+    }
+#pragma unroll
+    for (int i = 8; i < BN; ++i) mx[i & 7] = fminf(mx[i & 7], __uint_as_float(s[i]));
+    return fminf(fminf(fminf(mx[0], mx[1]), fminf(mx[2], mx[3])),
+                 fminf(fminf(mx[4], mx[5]), fminf(mx[6], mx[7]))) * sl2;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < BN; ++i) {
+      const float v = i < nvalid ? __uint_as_float(s[i]) * sl2 : -INFINITY;
+      s[i] = __float_as_uint(v);
+      mx[i & 7] = fmaxf(mx[i & 7], v);
+    }
+    return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+  }
+}
+
+// P = exp2(s·scale·log2e − mref) for this thread's row, rounded to 16 bits and
+// written over S in TMEM (four 16-column quarters); returns the sums of the
+// rounded and of the unrounded P.
+template <bool BF16, bool MASKED>
+__device__ __forceinline__ void exp_store(const uint32_t (&s)[BN], float sl2, float mref,
+                                          uint32_t t_p, float& lsum_r, float& lsum_e) {
+  float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc_e[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int col = 32 * h + 2 * i;
+      float p0, p1;
+      if constexpr (!MASKED) {
+        p0 = ex2_approx(fmaf(__uint_as_float(s[col]), sl2, -mref));
+        p1 = ex2_approx(fmaf(__uint_as_float(s[col + 1]), sl2, -mref));
+      } else {
+        p0 = ex2_approx(__uint_as_float(s[col]) - mref);
+        p1 = ex2_approx(__uint_as_float(s[col + 1]) - mref);
+      }
+      pk[i] = pack2<BF16>(p0, p1, acc[i & 3], acc_e[i & 3]);
+    }
+    tmem_st_x16(t_p + 16 * h, pk);
+  }
+  lsum_r = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  lsum_e = (acc_e[0] + acc_e[1]) + (acc_e[2] + acc_e[3]);
+}
+
+template <int D, bool BF16>
+__device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uint32_t tmem,
+                             const Ctl& c, int t) {
+  using L = Layout<D>;
+  const int r = threadIdx.x & 127;                           // row within the Q tile
+  const uint32_t lane_base = (uint32_t)((threadIdx.x >> 5) & 3) * 32;
+  const uint32_t t_s = tmem + (lane_base << 16) + S_COL[t];  // this warp's lanes of S_t / P_t
+  float* alpha_s = reinterpret_cast<float*>(smem + L::OFF_ALPHA) + t * BM;
+  float4* stats = reinterpret_cast<float4*>(smem + L::OFF_STATS);
+  const float sl2 = p.scale_log2;
+  uint32_t sf_ph = 0;
+  int units_done = 0;
+  Unit U;
+  for (int it = 0; next_unit(p, it, U); ++it) {
+    if (U.n[t] == 0) continue;
+    const int row = U.mb[t] * BM + r;
+    // l_r: sum of the rounded P (normalises O, matching what P·V consumed);
+    // l_e: sum of the unrounded P (gives LSE).
+    float m = -INFINITY, l_r = 0.f, l_e = 0.f;
+    for (int j = 0; j < U.n[t]; ++j) {
+      if (!wait_bar_warp(bar_addr<D>(sbase, BAR_SFULL + t), sf_ph, c)) return;
+      sf_ph ^= 1;
+      tc_fence_after();
+      uint32_t s[BN];
+#pragma unroll
+      for (int q = 0; q < BN / 32; ++q) tmem_ld_x32(t_s + 32 * q, s + 32 * q);
+      tmem_wait_ld();
+#pragma unroll
+      for (int q = 0; q < BN / 32; ++q) reg_pin_x32(s + 32 * q);
+
+      const bool masked = tile_needs_mask(p.s, U, t, j);
+      int nvalid = 0;
+      if (masked) {
+        int limit = U.key_len;
+        if (p.s.causal) limit = min(limit, row + 1);
+        nvalid = limit - j * BN;  // keys c < nvalid of this tile are allowed
+      }
+      const float m_cand = masked ? row_max<true>(s, sl2, nvalid) : row_max<false>(s, sl2, 0);
+      // Keep the old reference max unless the new one is RESCALE_THRESHOLD
+      // (log2) above it: O and l share the reference, so the result is
+      // unchanged, P stays below 2^8 and the O rescale is skipped.
+      const float m_new = (m_cand > m + RESCALE_THRESHOLD) ? m_cand : m;
+      const float alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
+      if (j > 0) {
+        alpha_s[r] = alpha;
+        mbar_arrive(bar_addr<D>(sbase, BAR_AFULL + t));
+      }
+      m = m_new;
+      const float mref = (m == -INFINITY) ? 0.f : m;
+      float lsum_r, lsum_e;
+      if (masked) exp_store<BF16, true>(s, sl2, mref, t_s, lsum_r, lsum_e);
+      else exp_store<BF16, false>(s, sl2, mref, t_s, lsum_r, lsum_e);
+      tmem_wait_st();
+      l_r = l_r * alpha + lsum_r;
+      l_e = l_e * alpha + lsum_e;
+      tc_fence_before();
+      mbar_arrive(bar_addr<D>(sbase, BAR_PFULL + t));
+    }
+    // One barrier per stats buffer: buffer (k & 1) is rewritten only after
+    // the epilogue of unit k has read it (the next-but-one unit's first P·V
+    // waits for that epilogue to free O), so no barrier runs a phase ahead.
+    const int buf = units_done & 1;
+    stats[(buf * 2 + t) * BM + r] = make_float4(m, l_r, l_e, 0.f);
+    ++units_done;
+    mbar_arrive(bar_addr<D>(sbase, BAR_STATS + 2 * t + buf));
+  }
+}
+
+// ====================================================== correction/epilogue
+template <int D, bool BF16>
+__device__ __forceinline__ uint32_t cvt2(float lo, float hi) {
+  if constexpr (BF16) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  } else {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+template <int D, bool BF16>
+__device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, uint32_t tmem,
+                                const Ctl& c, const CUtensorMap* tm_o) {
+  using L = Layout<D>;
+  const int r = threadIdx.x & 127;
+  const int wl = (threadIdx.x >> 5) & 3;  // warp within the group = 32-row slab
+  const int lane = threadIdx.x & 31;
+  const uint32_t lane_base = (uint32_t)wl * 32;
+  const float* alpha_all = reinterpret_cast<const float*>(smem + L::OFF_ALPHA);
+  const float4* stats = reinterpret_cast<const float4*>(smem + L::OFF_STATS);
+  uint32_t af_ph[2] = {0, 0}, pv_ph[2] = {0, 0};
+  int units_done[2] = {0, 0};
+  int ost = 0;  // staging buffer toggle (per warp)
+  bool ok = true;
+  Unit U;
+  for (int it = 0; ok && next_unit(p, it, U); ++it) {
+    // ---- rescale O_t for every K/V tile after the first
+    for (int j = 1; j < U.nmax && ok; ++j) {
+      for (int t = 0; t < 2; ++t) {
+        if (j >= U.n[t]) continue;
+        if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_AFULL + t), af_ph[t], c))) break;
+        af_ph[t] ^= 1;
+        const float a = alpha_all[t * BM + r];
+        if (__any_sync(0xffffffffu, a != 1.f)) {
+          tc_fence_after();
+          const uint32_t t_o = tmem + (lane_base << 16) + TmemO<D>::col(t);
+#pragma unroll 1
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t o[32];
+            tmem_ld_x32(t_o + 32 * q, o);
+            tmem_wait_ld();
+            reg_pin_x32(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * a);
+            tmem_st_x32(t_o + 32 * q, o);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(bar_addr<D>(sbase, BAR_OCORR + t));
+      }
+    }
+    if (!ok) break;
+    // ---- epilogue: O / l -> 16-bit -> smem (64-byte swizzle) -> TMA store; LSE
+    for (int t = 0; t < 2 && ok; ++t) {
+      if (!U.present[t]) continue;
+      const int row = U.mb[t] * BM + r;
+      const int head = U.b * p.s.Hq + U.hq[t];
+      float inv_l = 0.f, lse = -INFINITY;
+      const bool has = U.n[t] > 0;
+      if (has) {
+        const int k = units_done[t]++, buf = k & 1;
+        if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_STATS + 2 * t + buf), (k >> 1) & 1, c)))
+          break;
+        const float4 ml = stats[(buf * 2 + t) * BM + r];
+        if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_PVDONE + t), pv_ph[t], c))) break;
+        pv_ph[t] ^= 1;
+        tc_fence_after();
+        if (ml.y > 0.f) {
+          inv_l = 1.f / ml.y;
+          lse = (ml.x + log2f(ml.z)) * 0.69314718055994531f;
+        }
+      }
+      const int slab_row0 = U.mb[t] * BM + 32 * wl;
+      const uint32_t t_o = tmem + (lane_base << 16) + TmemO<D>::col(t);
+#pragma unroll 1
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t o[32];
+        if (has) {
+          tmem_ld_x32(t_o + 32 * q, o);
+          tmem_wait_ld();
+          reg_pin_x32(o);
+          if (q == D / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(bar_addr<D>(sbase, BAR_OFREE + t));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = cvt2<D, BF16>(__uint_as_float(o[2 * i]) * inv_l,
+                                __uint_as_float(o[2 * i + 1]) * inv_l);
+        uint8_t* buf = smem + L::OFF_OST + (wl * 2 + ost) * OST_BYTES;
+        if (lane == 0) bulk_wait_group_read<1>();  // the store that used `buf` last has read it
+        __syncwarp();
+        // row `lane`, 16-byte chunk k lands at chunk k ^ ((row >> 1) & 3): 64-byte swizzle
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint4 v = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+          *reinterpret_cast<uint4*>(buf + lane * 64 + ((k ^ ((lane >> 1) & 3)) * 16)) = v;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && slab_row0 < p.s.N) {
+          tma_store_3d(tm_o, smem_addr(buf), 32 * q, slab_row0, head);
+          bulk_commit_group();
+        }
+        ost ^= 1;
+      }
+      if (p.lse != nullptr && row < p.s.N) p.lse[(size_t)head * p.s.N + row] = lse;
+    }
+  }
+  if (lane == 0) bulk_wait_group<0>();
+  __syncwarp();
+}
+
+// ================================================================== kernel
+template <int D, bool BF16>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const Params p) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_addr<D>(sbase, BAR_QFULL + t), 1);
+      mbar_init(bar_addr<D>(sbase, BAR_QEMPTY + t), 1);
+      mbar_init(bar_addr<D>(sbase, BAR_SFULL + t), 1);
+      mbar_init(bar_addr<D>(sbase, BAR_PFULL + t), BM);
+      mbar_init(bar_addr<D>(sbase, BAR_AFULL + t), BM);
+      mbar_init(bar_addr<D>(sbase, BAR_OCORR + t), BM);
+      mbar_init(bar_addr<D>(sbase, BAR_PVDONE + t), 1);
+      mbar_init(bar_addr<D>(sbase, BAR_OFREE + t), BM);
+      mbar_init(bar_addr<D>(sbase, BAR_STATS + 2 * t), BM);
+      mbar_init(bar_addr<D>(sbase, BAR_STATS + 2 * t + 1), BM);
+    }
+    mbar_init(bar_addr<D>(sbase, BAR_DRAIN), 1);
+    for (int s = 0; s < L::STAGES; ++s) {
+      mbar_init(bar_addr<D>(sbase, BAR_KV + s), 1);
+      mbar_init(bar_addr<D>(sbase, BAR_KV + L::STAGES + s), 1);
+    }
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 12) {
+    tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 13 && lane == 0) {
+    tma_prefetch_map(&tm_q);
+    tma_prefetch_map(&tm_k);
+    tma_prefetch_map(&tm_v);
+    tma_prefetch_map(&tm_o);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Ctl ctl{abort_flag, p.timeout_ns};
+
+  // Register split: 2×192 (softmax) + 80 (correction) + 48 (MMA, loads) = 4 × 128.
+  if (warp < 8) {
+    setmaxnreg_inc<192>();
+    role_softmax<D, BF16>(p, smem, sbase, tmem, ctl, warp >> 2);
+  } else if (warp < 12) {
+    setmaxnreg_dec<80>();
+    role_correction<D, BF16>(p, smem, sbase, tmem, ctl, &tm_o);
+  } else {
+    setmaxnreg_dec<48>();
+    if (warp == 12 && lane == 0) role_mma<D, BF16>(p, sbase, tmem, ctl);
+    if (warp == 13 && lane == 0) role_load<D>(p, sbase, ctl, &tm_q, &tm_k, &tm_v);
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 12) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Bounded-wait self test: one thread waits on a barrier nothing arrives at.
+__global__ void fa_wait_selftest_kernel(unsigned long long timeout_ns, int* out) {
+  __shared__ alignas(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_addr(&bar), 1);
+    mbar_init_fence();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    Ctl c{&abort_flag, timeout_ns};
+    const bool ok = wait_bar(smem_addr(&bar), 0, c);
+    out[0] = ok ? 1 : 0;
+    out[1] = abort_flag;
+  }
+}
+
+}  // namespace fa
+
+// ==================================================================== host
+namespace {
+
+thread_local char g_err[512] = "";
+unsigned long long g_timeout_ns = 4000ull * 1000000ull;
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+using AddressRangeFn = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+struct DriverFns {
+  EncodeTiledFn encode = nullptr;
+  AddressRangeFn range = nullptr;
+  bool ok = false;
+};
+
+const DriverFns& driver_fns() {
+  static DriverFns fns;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q1, q2;
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f1, 12000, cudaEnableDefault,
+                                         &q1) == cudaSuccess &&
+        q1 == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &f2, 12000, cudaEnableDefault,
+                                         &q2) == cudaSuccess &&
+        q2 == cudaDriverEntryPointSuccess) {
+      fns.encode = reinterpret_cast<EncodeTiledFn>(f1);
+      fns.range = reinterpret_cast<AddressRangeFn>(f2);
+      fns.ok = true;
+    }
+  });
+  return fns;
+}
+
+struct DeviceInfo {
+  bool init = false;
+  bool sm100 = false;
+  int sms = 0;
+  bool attr_set[4] = {false, false, false, false};
+};
+DeviceInfo g_dev[64];
+std::mutex g_dev_mu;
+
+// [ptr, ptr + bytes) must lie inside one device allocation of the current device.
+int check_range(const char* name, const void* ptr, size_t bytes, size_t align) {
+  if (ptr == nullptr) return fail(FA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (reinterpret_cast<uintptr_t>(ptr) % align != 0)
+    return fail(FA_ERR_INVALID_ARG, "%s is not %zu-byte aligned", name, align);
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FA_ERR_INVALID_ARG, "%s is not a CUDA pointer", name);
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+    return fail(FA_ERR_INVALID_ARG, "%s is not device memory", name);
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (a.device != dev) return fail(FA_ERR_INVALID_ARG, "%s lives on device %d, not %d", name, a.device, dev);
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (driver_fns().range(&base, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS)
+    return fail(FA_ERR_INVALID_ARG, "%s: no allocation found", name);
+  const uintptr_t p = reinterpret_cast<uintptr_t>(ptr);
+  if (p + bytes > static_cast<uintptr_t>(base) + size)
+    return fail(FA_ERR_INVALID_ARG, "%s: %zu bytes run past its allocation", name, bytes);
+  return FA_OK;
+}
+
+int make_map(CUtensorMap* map, const void* ptr, bool bf16, int d, int n, long long heads,
+             int box_cols, int box_rows, CUtensorMapSwizzle swz) {
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)heads};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * (cuuint64_t)n};
+  const cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = driver_fns().encode(
+      map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+      const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return FA_OK;
+}
+
+template <int D, bool BF16>
+int launch(const void* q, const void* k, const void* v, void* o, const fa::Params& prm,
+           cudaStream_t stream, DeviceInfo& info, int slot) {
+  using L = fa::Layout<D>;
+  auto kern = fa::fa_fwd_kernel<D, BF16>;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!info.attr_set[slot]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) !=
+          cudaSuccess)
+        return fail(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
+      cudaFuncAttributes fa_attr;
+      if (cudaFuncGetAttributes(&fa_attr, kern) != cudaSuccess)
+        return fail(FA_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(cudaGetLastError()));
+      // The setmaxnreg split (2×192 + 80 + 48 per 128 threads) needs exactly 128
+      // registers per thread at launch; anything else could never be satisfied.
+      if (fa_attr.numRegs != 128)
+        return fail(FA_ERR_UNSUPPORTED, "kernel built with %d registers per thread, need 128",
+                    fa_attr.numRegs);
+      info.attr_set[slot] = true;
+    }
+  }
+  CUtensorMap tq, tk, tv, to;
+  const fa::Shape& s = prm.s;
+  int rc;
+  if ((rc = make_map(&tq, q, BF16, D, s.N, (long long)s.B * s.Hq, 64, fa::BM,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
+  if ((rc = make_map(&tk, k, BF16, D, s.N, (long long)s.B * s.Hk, 64, fa::BN,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
+  if ((rc = make_map(&tv, v, BF16, D, s.N, (long long)s.B * s.Hk, 64, fa::BN,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
+  if ((rc = make_map(&to, o, BF16, D, s.N, (long long)s.B * s.Hq, 32, 32,
+                     CU_TENSOR_MAP_SWIZZLE_64B)) != FA_OK) return rc;
+  const int grid = s.num_units < info.sms ? s.num_units : info.sms;
+  kern<<<grid, fa::NUM_THREADS, L::ALLOC, stream>>>(tq, tk, tv, to, prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return 100; }
+
+const char* fa_last_error_string(void) { return g_err; }
+
+int fa_set_wait_timeout_ms(int ms) {
+  if (ms < 1 || ms > 600000) return fail(FA_ERR_INVALID_ARG, "timeout %d ms out of [1, 600000]", ms);
+  g_timeout_ns = (unsigned long long)ms * 1000000ull;
+  return FA_OK;
+}
+
+int fa_num_units(int B, int Hq, int Hk, int N, int causal) {
+  if (B < 1 || Hq < 1 || Hk < 1 || N < 1 || Hq % Hk != 0)
+    return fail(FA_ERR_INVALID_ARG, "bad shape");
+  const long long units = (long long)B * Hk * ((((long long)Hq / Hk) * ((N + 127) / 128) + 1) / 2);
+  if (units > 0x7fffffffLL) return fail(FA_ERR_INVALID_ARG, "too many work units");
+  return fa::make_shape(B, Hq, Hk, N, causal).num_units;
+}
+
+int fa_unit_info(int B, int Hq, int Hk, int N, int causal, int u, int32_t* out) {
+  const int nu = fa_num_units(B, Hq, Hk, N, causal);
+  if (nu < 0) return nu;
+  if (out == nullptr || u < 0 || u >= nu) return fail(FA_ERR_INVALID_ARG, "bad unit index");
+  fa::Unit U;
+  fa::decode_unit(fa::make_shape(B, Hq, Hk, N, causal), u, U);
+  const int32_t vals[8] = {U.b, U.hk, U.hq[0], U.mb[0], U.present[0], U.hq[1], U.mb[1], U.present[1]};
+  memcpy(out, vals, sizeof(vals));
+  return FA_OK;
+}
+
+int fa_unit_for(int cta, int it, int grid) { return fa::unit_for(cta, it, grid); }
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hk,
+           int N, int d, float scale, int causal, const int32_t* key_pad_lens, void* stream,
+           int dtype) {
+  g_err[0] = '\0';
+  // ---- arguments that need no CUDA call
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr)
+    return fail(FA_ERR_INVALID_ARG, "q, k, v and o must be non-NULL");
+  if (B < 1 || Hq < 1 || Hk < 1 || N < 1)
+    return fail(FA_ERR_INVALID_ARG, "B, Hq, Hk and N must be >= 1");
+  if (Hq % Hk != 0) return fail(FA_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hk (%d)", Hq, Hk);
+  if (d != 64 && d != 128)
+    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", d);
+  if (dtype != FA_FP16 && dtype != FA_BF16) return fail(FA_ERR_UNSUPPORTED, "unknown dtype %d", dtype);
+  if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "scale must be finite");
+  if (causal != 0 && causal != 1) return fail(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  const long long heads_q = (long long)B * Hq, heads_k = (long long)B * Hk;
+  if (heads_q > 0x7fffffffLL || N > (1 << 30))
+    return fail(FA_ERR_INVALID_ARG, "problem too large for 32-bit tile coordinates");
+  if (fa_num_units(B, Hq, Hk, N, causal) < 0) return FA_ERR_INVALID_ARG;
+  // ---- device and buffers
+  if (!driver_fns().ok) return fail(FA_ERR_CUDA, "CUDA driver entry points unavailable");
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return fail(FA_ERR_CUDA, "no current CUDA device");
+  DeviceInfo& info = g_dev[dev];
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!info.init) {
+      cudaDeviceProp prop;
+      if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess)
+        return fail(FA_ERR_CUDA, "cudaGetDeviceProperties failed");
+      info.sm100 = prop.major == 10 && prop.minor == 0;
+      info.sms = prop.multiProcessorCount;
+      info.init = true;
+    }
+  }
+  if (!info.sm100) return fail(FA_ERR_UNSUPPORTED, "device %d is not sm_100", dev);
+  const size_t q_bytes = (size_t)heads_q * N * d * 2, kv_bytes = (size_t)heads_k * N * d * 2;
+  int rc;
+  if ((rc = check_range("q", q, q_bytes, 16)) != FA_OK) return rc;
+  if ((rc = check_range("k", k, kv_bytes, 16)) != FA_OK) return rc;
+  if ((rc = check_range("v", v, kv_bytes, 16)) != FA_OK) return rc;
+  if ((rc = check_range("o", o, q_bytes, 16)) != FA_OK) return rc;
+  if (lse != nullptr && (rc = check_range("lse", lse, (size_t)heads_q * N * 4, 4)) != FA_OK) return rc;
+  if (key_pad_lens != nullptr &&
+      (rc = check_range("key_pad_lens", key_pad_lens, (size_t)B * 4, 4)) != FA_OK)
+    return rc;
+  const uintptr_t ob = reinterpret_cast<uintptr_t>(o), oe = ob + q_bytes;
+  auto overlaps = [&](const void* x, size_t n) {
+    const uintptr_t xb = reinterpret_cast<uintptr_t>(x);
+    return xb < oe && ob < xb + n;
+  };
+  if (overlaps(q, q_bytes) || overlaps(k, kv_bytes) || overlaps(v, kv_bytes) ||
+      (lse != nullptr && overlaps(lse, (size_t)heads_q * N * 4)))
+    return fail(FA_ERR_INVALID_ARG, "o overlaps an input or lse");
+
+  fa::Params prm;
+  prm.key_pad_lens = key_pad_lens;
+  prm.lse = lse;
+  prm.s = fa::make_shape(B, Hq, Hk, N, causal);
+  prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  prm.timeout_ns = g_timeout_ns;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == FA_BF16;
+  if (d == 128)
+    return bf16 ? launch<128, true>(q, k, v, o, prm, st, info, 0)
+                : launch<128, false>(q, k, v, o, prm, st, info, 1);
+  return bf16 ? launch<64, true>(q, k, v, o, prm, st, info, 2)
+              : launch<64, false>(q, k, v, o, prm, st, info, 3);
+}
+
+int fa_get_device_status(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess)
+    return fail(FA_ERR_CUDA, "cudaDeviceSynchronize: %s", cudaGetErrorString(cudaGetLastError()));
+  int status = 0;
+  if (cudaMemcpyFromSymbol(&status, fa::g_fa_status, sizeof(int)) != cudaSuccess)
+    return fail(FA_ERR_CUDA, "reading the status word failed");
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(int)) != cudaSuccess)
+    return fail(FA_ERR_CUDA, "clearing the status word failed");
+  return status;
+}
+
+// Runs the bounded wait on a barrier that nothing arrives at, with a limit of
+// `ms` milliseconds; returns FA_OK when the wait gave up as designed (and
+// leaves FA_ERR_DEVICE_TIMEOUT in the status word).
+int fa_selftest_wait_timeout(int ms) {
+  if (ms < 1 || ms > 10000) return fail(FA_ERR_INVALID_ARG, "ms out of [1, 10000]");
+  int* d_out = nullptr;
+  if (cudaMalloc(&d_out, 2 * sizeof(int)) != cudaSuccess) return fail(FA_ERR_CUDA, "cudaMalloc");
+  fa::fa_wait_selftest_kernel<<<1, 32>>>((unsigned long long)ms * 1000000ull, d_out);
+  int h[2] = {-1, -1};
+  cudaError_t e = cudaMemcpy(h, d_out, sizeof(h), cudaMemcpyDeviceToHost);
+  cudaFree(d_out);
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "self test: %s", cudaGetErrorString(e));
+  if (h[0] != 0 || h[1] != 1) return fail(FA_ERR_CUDA, "self test: wait did not give up");
+  return FA_OK;
+}
+
+}  // extern "C"
