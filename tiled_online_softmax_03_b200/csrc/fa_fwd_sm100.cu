@@ -220,129 +220,143 @@ __device__ void role_load(const Params& p, uint32_t sbase, const Ctl& c, const C
 }
 
 // ============================================================= MMA issuer
+// Run by the whole of warp 12, converged; one elected lane issues each
+// tcgen05 instruction.
 template <int D, bool BF16>
 __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const Ctl& c) {
   using L = Layout<D>;
   constexpr uint32_t IDESC_QK = idesc_f16(BF16, BN, false);  // S = Q·Kᵀ, both K-major
   constexpr uint32_t IDESC_PV = idesc_f16(BF16, D, true);    // O += P·V, V is MN-major
-  uint32_t qf_ph[2] = {0, 0}, pf_ph[2] = {0, 0}, oc_ph[2] = {0, 0}, of_ph[2] = {0, 0};
   int st = 0;
   uint32_t kv_ph = 0;
   bool ok = true;
 
-  // Descriptors are built once per operand tile; a K step adds its byte
-  // offset >> 4 to the start-address field (bits 0-13, no carry out: < 256 KB).
+  // Issue cost matters as much as tensor time here: one 128x128x16 MMA runs
+  // in ~64 cycles, so each issue must be a handful of instructions. The K
+  // loops are unrolled with compile-time offsets added to a descriptor built
+  // once per call (a K step adds its byte offset >> 4 to the start-address
+  // field, bits 0-13, with no carry out since shared memory is < 256 KB), and
+  // the accumulate flag is a compile-time constant except on the first step.
+  const uint64_t q_desc0 = sdesc(sbase + L::OFF_Q, 16, 1024);
+  const uint64_t kv_desc0 = sdesc(sbase + L::OFF_KV, 16, 1024);
+  const uint64_t v_desc0 = sdesc(sbase + L::OFF_KV, SW128_BOX_BYTES, 1024);
   auto issue_qk = [&](int t, int kst) {
-    const uint64_t qd = sdesc(sbase + L::OFF_Q + t * L::Q_BYTES, 16, 1024);
-    const uint64_t kd = sdesc(sbase + L::OFF_KV + kst * L::KV_BYTES, 16, 1024);
+    const uint64_t qd = q_desc0 + (uint64_t)((t * L::Q_BYTES) >> 4);
+    const uint64_t kd = kv_desc0 + (uint64_t)((kst * L::KV_BYTES) >> 4);
     const uint32_t d_s = tmem + S_COL[t];
-#pragma unroll 1
-    for (int k = 0; k < D / 16; ++k) {
+    umma_ss_warp(d_s, qd, kd, IDESC_QK, 0u);
+#pragma unroll
+    for (int k = 1; k < D / 16; ++k) {
       const uint32_t off = ((k >> 2) * SW128_BOX_BYTES + (k & 3) * 32) >> 4;
-      umma_ss(d_s, qd + off, kd + off, IDESC_QK, k > 0);
+      umma_ss_warp(d_s, qd + off, kd + off, IDESC_QK, 1u);
     }
   };
-  auto issue_pv = [&](int t, int vst, bool acc) {
+  auto issue_pv = [&](int t, int vst, uint32_t acc) {
     // P: 16 keys = 8 TMEM columns (two 16-bit values per column); V: 16 key
     // rows of 128 bytes in each 64-column box, boxes SW128_BOX_BYTES apart.
-    const uint64_t vd = sdesc(sbase + L::OFF_KV + vst * L::KV_BYTES, SW128_BOX_BYTES, 1024);
+    const uint64_t vd = v_desc0 + (uint64_t)((vst * L::KV_BYTES) >> 4);
     const uint32_t d_o = tmem + TmemO<D>::col(t);
     const uint32_t a_p = tmem + S_COL[t];
-#pragma unroll 1
-    for (int k = 0; k < BN / 16; ++k)
-      umma_ts(d_o, a_p + k * 8, vd + ((k * 16 * 128) >> 4), IDESC_PV, (acc || k > 0) ? 1u : 0u);
+    umma_ts_warp(d_o, a_p, vd, IDESC_PV, acc);
+#pragma unroll
+    for (int k = 1; k < BN / 16; ++k)
+      umma_ts_warp(d_o, a_p + k * 8, vd + ((k * 16 * 128) >> 4), IDESC_PV, 1u);
   };
 
+  // Phase bits, one per barrier the MMA thread waits on.
+  constexpr uint32_t QF = 0, PF = 2, OC = 4, OF = 6;
+  uint32_t ph = 0;
+  auto wait_flip = [&](int bar, uint32_t bit, uint32_t invert) {
+    const bool r = wait_bar_warp(bar_addr<D>(sbase, bar), ((ph >> bit) & 1u) ^ invert, c);
+    ph ^= 1u << bit;
+    return r;
+  };
   Unit U;
   for (int it = 0; ok && next_unit(p, it, U); ++it) {
-    if (U.nmax == 0) continue;
+    const int n0 = U.n[0], n1 = U.n[1], nmax = U.nmax;
+    if (nmax == 0) continue;
     const int k0 = st;
     const uint32_t k0_ph = kv_ph;
     if (++st == L::STAGES) { st = 0; kv_ph ^= 1; }
-    if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_KV + k0), k0_ph, c))) break;
-    for (int t = 0; t < 2 && ok; ++t) {
-      if (U.n[t] == 0) continue;
-      if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_QFULL + t), qf_ph[t], c))) break;
-      qf_ph[t] ^= 1;
-    }
-    if (!ok) break;
+    if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_KV + k0), k0_ph, c))) break;
+    if (n0 > 0 && !(ok = wait_flip(BAR_QFULL + 0, QF + 0, 0))) break;
+    if (n1 > 0 && !(ok = wait_flip(BAR_QFULL + 1, QF + 1, 0))) break;
     tc_fence_after();
-    for (int t = 0; t < 2; ++t) {
-      if (U.n[t] == 0) continue;
-      issue_qk(t, k0);
-      umma_commit(bar_addr<D>(sbase, BAR_SFULL + t));
+    if (n0 > 0) {
+      issue_qk(0, k0);
+      umma_commit_warp(bar_addr<D>(sbase, BAR_SFULL + 0));
     }
-    umma_commit(bar_addr<D>(sbase, BAR_KV + L::STAGES + k0));
+    if (n1 > 0) {
+      issue_qk(1, k0);
+      umma_commit_warp(bar_addr<D>(sbase, BAR_SFULL + 1));
+    }
+    umma_commit_warp(bar_addr<D>(sbase, BAR_KV + L::STAGES + k0));
 
-    for (int j = 0; j < U.nmax && ok; ++j) {
+    for (int j = 0; j < nmax && ok; ++j) {
       const int vs = st;
       const uint32_t vs_ph = kv_ph;
       if (++st == L::STAGES) { st = 0; kv_ph ^= 1; }
       int kn = -1;
       uint32_t kn_ph = 0;
-      if (j + 1 < U.nmax) {
+      if (j + 1 < nmax) {
         kn = st;
         kn_ph = kv_ph;
         if (++st == L::STAGES) { st = 0; kv_ph ^= 1; }
       }
-      if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_KV + vs), vs_ph, c))) break;
+      if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_KV + vs), vs_ph, c))) break;
       bool kn_ready = false;
       for (int t = 0; t < 2; ++t) {
-        if (j >= U.n[t]) continue;
-        if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_PFULL + t), pf_ph[t], c))) break;
-        pf_ph[t] ^= 1;
+        const int nt = t ? n1 : n0;
+        if (j >= nt) continue;
+        if (!(ok = wait_flip(BAR_PFULL + t, PF + t, 0))) break;
         if (j > 0) {
-          if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_OCORR + t), oc_ph[t], c))) break;
-          oc_ph[t] ^= 1;
+          if (!(ok = wait_flip(BAR_OCORR + t, OC + t, 0))) break;
         } else {
-          if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_OFREE + t), of_ph[t] ^ 1, c))) break;
-          of_ph[t] ^= 1;
+          if (!(ok = wait_flip(BAR_OFREE + t, OF + t, 1))) break;
         }
         tc_fence_after();
-        issue_pv(t, vs, j > 0);
-        if (j == U.n[t] - 1) {
-          umma_commit(bar_addr<D>(sbase, BAR_PVDONE + t));
-          umma_commit(bar_addr<D>(sbase, BAR_QEMPTY + t));
+        issue_pv(t, vs, j > 0 ? 1u : 0u);
+        if (j == nt - 1) {
+          umma_commit_warp(bar_addr<D>(sbase, BAR_PVDONE + t));
+          umma_commit_warp(bar_addr<D>(sbase, BAR_QEMPTY + t));
         } else {
           if (!kn_ready) {
-            if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_KV + kn), kn_ph, c))) break;
+            if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_KV + kn), kn_ph, c))) break;
             kn_ready = true;
             tc_fence_after();
           }
           issue_qk(t, kn);
-          umma_commit(bar_addr<D>(sbase, BAR_SFULL + t));
+          umma_commit_warp(bar_addr<D>(sbase, BAR_SFULL + t));
         }
       }
       if (!ok) break;
-      umma_commit(bar_addr<D>(sbase, BAR_KV + L::STAGES + vs));
-      if (kn >= 0) umma_commit(bar_addr<D>(sbase, BAR_KV + L::STAGES + kn));
+      umma_commit_warp(bar_addr<D>(sbase, BAR_KV + L::STAGES + vs));
+      if (kn >= 0) umma_commit_warp(bar_addr<D>(sbase, BAR_KV + L::STAGES + kn));
     }
   }
   if (!ok) {
     // Let every issued MMA finish before TMEM is released.
     volatile int no_abort = 0;
     Ctl drain{&no_abort, 100000000ull};
-    umma_commit(bar_addr<D>(sbase, BAR_DRAIN));
-    wait_bar(bar_addr<D>(sbase, BAR_DRAIN), 0, drain);
+    umma_commit_warp(bar_addr<D>(sbase, BAR_DRAIN));
+    wait_bar_warp(bar_addr<D>(sbase, BAR_DRAIN), 0, drain);
   }
 }
 
 // ================================================================= softmax
 // Rounds (lo, hi) to the 16-bit MMA type and packs them as one TMEM column
-// (lo in the low half). `sum_r` accumulates the rounded values (what the P·V
-// product consumes), `sum_e` the unrounded ones.
+// (lo in the low half); also returns the two rounded values as fp32.
 template <bool BF16>
-__device__ __forceinline__ uint32_t pack2(float lo, float hi, float& sum_r, float& sum_e) {
-  sum_e += lo + hi;
+__device__ __forceinline__ uint32_t round_pack(float lo, float hi, uint64_t& rounded) {
   if constexpr (BF16) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    const float2 f = __bfloat1622float2(h);
-    sum_r += f.x + f.y;
-    return *reinterpret_cast<uint32_t*>(&h);
+    const uint32_t u = *reinterpret_cast<uint32_t*>(&h);
+    rounded = ((uint64_t)(u & 0xffff0000u) << 32) | (uint64_t)(u << 16);  // bf16 -> fp32 is a shift
+    return u;
   } else {
     __half2 h = __floats2half2_rn(lo, hi);
     const float2 f = __half22float2(h);
-    sum_r += f.x + f.y;
+    rounded = f2_pack(f.x, f.y);
     return *reinterpret_cast<uint32_t*>(&h);
   }
 }
@@ -359,55 +373,57 @@ __device__ __forceinline__ float row_max(uint32_t (&s)[BN], float sl2, int nvali
     for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(s[i]);
     if (sl2 >= 0.f) {
 #pragma unroll
-      for (int i = 8; i < BN; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(s[i]));
-      return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+      for (int i = 8; i < BN; i += 2)
+        mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
+      return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl2;
     }
 #pragma unroll
-    for (int i = 8; i < BN; ++i) mx[i & 7] = fminf(mx[i & 7], __uint_as_float(s[i]));
-    return fminf(fminf(fminf(mx[0], mx[1]), fminf(mx[2], mx[3])),
-                 fminf(fminf(mx[4], mx[5]), fminf(mx[6], mx[7]))) * sl2;
+    for (int i = 8; i < BN; i += 2)
+      mx[(i >> 1) & 7] = fmin3(mx[(i >> 1) & 7], __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
+    return fmin3(fmin3(mx[0], mx[1], mx[2]), fmin3(mx[3], mx[4], mx[5]), fminf(mx[6], mx[7])) * sl2;
   } else {
 #pragma unroll
     for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < BN; ++i) {
-      const float v = i < nvalid ? __uint_as_float(s[i]) * sl2 : -INFINITY;
-      s[i] = __float_as_uint(v);
-      mx[i & 7] = fmaxf(mx[i & 7], v);
+    for (int i = 0; i < BN; i += 2) {
+      const float v0 = i < nvalid ? __uint_as_float(s[i]) * sl2 : -INFINITY;
+      const float v1 = i + 1 < nvalid ? __uint_as_float(s[i + 1]) * sl2 : -INFINITY;
+      s[i] = __float_as_uint(v0);
+      s[i + 1] = __float_as_uint(v1);
+      mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], v0, v1);
     }
-    return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+    return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
   }
 }
 
 // P = exp2(s·scale·log2e − mref) for this thread's row, rounded to 16 bits and
-// written over S in TMEM (four 16-column quarters); returns the sums of the
-// rounded and of the unrounded P.
+// written over S in TMEM; returns the sums of the rounded and of the unrounded
+// P. The whole row is computed before the two TMEM stores so that the
+// exponentials of all 128 columns can overlap; scale-and-subtract and both
+// sums use packed fp32 pairs.
 template <bool BF16, bool MASKED>
 __device__ __forceinline__ void exp_store(const uint32_t (&s)[BN], float sl2, float mref,
                                           uint32_t t_p, float& lsum_r, float& lsum_e) {
-  float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc_e[4] = {0.f, 0.f, 0.f, 0.f};
+  const uint64_t k2 = f2_pack(sl2, sl2), nm2 = f2_pack(-mref, -mref);
+  uint64_t acc_r[4] = {0, 0, 0, 0}, acc_e[4] = {0, 0, 0, 0};
+  uint32_t pk[BN / 2];
 #pragma unroll
-  for (int h = 0; h < 4; ++h) {
-    uint32_t pk[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int col = 32 * h + 2 * i;
-      float p0, p1;
-      if constexpr (!MASKED) {
-        p0 = ex2_approx(fmaf(__uint_as_float(s[col]), sl2, -mref));
-        p1 = ex2_approx(fmaf(__uint_as_float(s[col + 1]), sl2, -mref));
-      } else {
-        p0 = ex2_approx(__uint_as_float(s[col]) - mref);
-        p1 = ex2_approx(__uint_as_float(s[col + 1]) - mref);
-      }
-      pk[i] = pack2<BF16>(p0, p1, acc[i & 3], acc_e[i & 3]);
-    }
-    tmem_st_x16(t_p + 16 * h, pk);
+  for (int i = 0; i < BN / 2; ++i) {
+    const uint64_t x = ((uint64_t)s[2 * i + 1] << 32) | s[2 * i];
+    const uint64_t y = MASKED ? fadd2(x, nm2) : ffma2(x, k2, nm2);
+    const float p0 = ex2_approx(f2_lo(y)), p1 = ex2_approx(f2_hi(y));
+    const uint64_t pp = f2_pack(p0, p1);
+    acc_e[i & 3] = fadd2(acc_e[i & 3], pp);
+    uint64_t rounded;
+    pk[i] = round_pack<BF16>(p0, p1, rounded);
+    acc_r[i & 3] = fadd2(acc_r[i & 3], rounded);
   }
-  lsum_r = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-  lsum_e = (acc_e[0] + acc_e[1]) + (acc_e[2] + acc_e[3]);
+  tmem_st_x32(t_p, pk);
+  tmem_st_x32(t_p + 32, pk + 32);
+  const uint64_t r2 = fadd2(fadd2(acc_r[0], acc_r[1]), fadd2(acc_r[2], acc_r[3]));
+  const uint64_t e2 = fadd2(fadd2(acc_e[0], acc_e[1]), fadd2(acc_e[2], acc_e[3]));
+  lsum_r = f2_lo(r2) + f2_hi(r2);
+  lsum_e = f2_lo(e2) + f2_hi(e2);
 }
 
 template <int D, bool BF16>
@@ -651,16 +667,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const Ctl ctl{abort_flag, p.timeout_ns};
 
-  // Register split: 2×192 (softmax) + 80 (correction) + 48 (MMA, loads) = 4 × 128.
+  // Register split: 2×176 (softmax) + 80 (correction) + 80 (MMA, loads) = 4 × 128.
   if (warp < 8) {
-    setmaxnreg_inc<192>();
+    setmaxnreg_inc<176>();
     role_softmax<D, BF16>(p, smem, sbase, tmem, ctl, warp >> 2);
   } else if (warp < 12) {
     setmaxnreg_dec<80>();
     role_correction<D, BF16>(p, smem, sbase, tmem, ctl, &tm_o);
   } else {
-    setmaxnreg_dec<48>();
-    if (warp == 12 && lane == 0) role_mma<D, BF16>(p, sbase, tmem, ctl);
+    setmaxnreg_dec<80>();
+    if (warp == 12) role_mma<D, BF16>(p, sbase, tmem, ctl);
     if (warp == 13 && lane == 0) role_load<D>(p, sbase, ctl, &tm_q, &tm_k, &tm_v);
     __syncwarp();
   }
@@ -802,7 +818,7 @@ int launch(const void* q, const void* k, const void* v, void* o, const fa::Param
       cudaFuncAttributes fa_attr;
       if (cudaFuncGetAttributes(&fa_attr, kern) != cudaSuccess)
         return fail(FA_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(cudaGetLastError()));
-      // The setmaxnreg split (2×192 + 80 + 48 per 128 threads) needs exactly 128
+      // The setmaxnreg split (2×176 + 80 + 80 per 128 threads) needs exactly 128
       // registers per thread at launch; anything else could never be satisfied.
       if (fa_attr.numRegs != 128)
         return fail(FA_ERR_UNSUPPORTED, "kernel built with %d registers per thread, need 128",
