@@ -345,21 +345,45 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
 
 // ================================================================= softmax
 // Rounds (lo, hi) to the 16-bit MMA type and packs them as one TMEM column
-// (lo in the low half); also returns the two rounded values as fp32.
+// (lo in the low half).
 template <bool BF16>
-__device__ __forceinline__ uint32_t round_pack(float lo, float hi, uint64_t& rounded) {
+__device__ __forceinline__ uint32_t round_pack(float lo, float hi) {
   if constexpr (BF16) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    const uint32_t u = *reinterpret_cast<uint32_t*>(&h);
-    rounded = ((uint64_t)(u & 0xffff0000u) << 32) | (uint64_t)(u << 16);  // bf16 -> fp32 is a shift
-    return u;
+    return *reinterpret_cast<uint32_t*>(&h);
   } else {
     __half2 h = __floats2half2_rn(lo, hi);
-    const float2 f = __half22float2(h);
-    rounded = f2_pack(f.x, f.y);
     return *reinterpret_cast<uint32_t*>(&h);
   }
 }
+
+// 2^y for a pair of fp32 values on the FMA pipe, relieving the MUFU pipe
+// (16 ex2 per clock per SM), which otherwise takes as long per K/V tile as
+// the tensor core at d = 128. Cody-Waite style reduction y = n + f with
+// n = round(y) (by adding 1.5·2^23, whose low mantissa bits then hold n) and
+// f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose coefficients minimise
+// the maximum relative error (Remez exchange, csrc/fit_exp2_poly.py: 7.5e-5,
+// below the 16-bit rounding that P gets next); 2^n is added to the exponent
+// field. Inputs are clamped to >= -126, where 2^y is far below any P that
+// survives 16-bit rounding next to the row's maximum.
+constexpr float EXP2_C0 = 9.999280572e-01f;
+constexpr float EXP2_C1 = 6.932609677e-01f;
+constexpr float EXP2_C2 = 2.426111251e-01f;
+constexpr float EXP2_C3 = 5.517166853e-02f;
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t y) {
+  const uint64_t yc = f2_pack(fmaxf(f2_lo(y), -126.f), fmaxf(f2_hi(y), -126.f));
+  const uint64_t t = fadd2(yc, f2_pack(12582912.f, 12582912.f));
+  const uint64_t n = fadd2(t, f2_pack(-12582912.f, -12582912.f));
+  const uint64_t f = ffma2(n, f2_pack(-1.f, -1.f), yc);
+  uint64_t q = ffma2(f2_pack(EXP2_C3, EXP2_C3), f, f2_pack(EXP2_C2, EXP2_C2));
+  q = ffma2(q, f, f2_pack(EXP2_C1, EXP2_C1));
+  q = ffma2(q, f, f2_pack(EXP2_C0, EXP2_C0));
+  const uint32_t r0 = (uint32_t)q + ((uint32_t)t << 23);
+  const uint32_t r1 = (uint32_t)(q >> 32) + ((uint32_t)(t >> 32) << 23);
+  return ((uint64_t)r1 << 32) | r0;
+}
+// One pair in every EXP2_FMA_EVERY takes the FMA-pipe exponential (unmasked tiles).
+constexpr int EXP2_FMA_EVERY = 1 << 30;  // off: measured slower here
 
 // Row max of one S tile for this thread's row, in log2 units of the scaled
 // score. MASKED: keys c >= nvalid are masked, and s is rewritten in place to
@@ -397,33 +421,42 @@ __device__ __forceinline__ float row_max(uint32_t (&s)[BN], float sl2, int nvali
 }
 
 // P = exp2(s·scale·log2e − mref) for this thread's row, rounded to 16 bits and
-// written over S in TMEM; returns the sums of the rounded and of the unrounded
-// P. The whole row is computed before the two TMEM stores so that the
-// exponentials of all 128 columns can overlap; scale-and-subtract and both
-// sums use packed fp32 pairs.
+// written over S in TMEM; returns the sum of the unrounded P. The whole row is
+// computed before the two TMEM stores so that the exponentials of all 128
+// columns can overlap; scale-and-subtract and the sum use packed fp32 pairs.
 template <bool BF16, bool MASKED>
-__device__ __forceinline__ void exp_store(const uint32_t (&s)[BN], float sl2, float mref,
-                                          uint32_t t_p, float& lsum_r, float& lsum_e) {
+__device__ __forceinline__ float exp_store(const uint32_t (&s)[BN], float sl2, float mref,
+                                           uint32_t t_p) {
   const uint64_t k2 = f2_pack(sl2, sl2), nm2 = f2_pack(-mref, -mref);
-  uint64_t acc_r[4] = {0, 0, 0, 0}, acc_e[4] = {0, 0, 0, 0};
+  uint64_t acc[4] = {0, 0, 0, 0};
   uint32_t pk[BN / 2];
 #pragma unroll
   for (int i = 0; i < BN / 2; ++i) {
     const uint64_t x = ((uint64_t)s[2 * i + 1] << 32) | s[2 * i];
     const uint64_t y = MASKED ? fadd2(x, nm2) : ffma2(x, k2, nm2);
-    const float p0 = ex2_approx(f2_lo(y)), p1 = ex2_approx(f2_hi(y));
-    const uint64_t pp = f2_pack(p0, p1);
-    acc_e[i & 3] = fadd2(acc_e[i & 3], pp);
-    uint64_t rounded;
-    pk[i] = round_pack<BF16>(p0, p1, rounded);
-    acc_r[i & 3] = fadd2(acc_r[i & 3], rounded);
+    float p0, p1;
+    if (!MASKED && i % EXP2_FMA_EVERY == EXP2_FMA_EVERY - 1) {
+      const uint64_t e = exp2_fma2(y);
+      p0 = f2_lo(e);
+      p1 = f2_hi(e);
+    } else {
+      p0 = ex2_approx(f2_lo(y));
+      p1 = ex2_approx(f2_hi(y));
+    }
+    acc[i & 3] = fadd2(acc[i & 3], f2_pack(p0, p1));
+    pk[i] = round_pack<BF16>(p0, p1);
   }
   tmem_st_x32(t_p, pk);
   tmem_st_x32(t_p + 32, pk + 32);
-  const uint64_t r2 = fadd2(fadd2(acc_r[0], acc_r[1]), fadd2(acc_r[2], acc_r[3]));
-  const uint64_t e2 = fadd2(fadd2(acc_e[0], acc_e[1]), fadd2(acc_e[2], acc_e[3]));
-  lsum_r = f2_lo(r2) + f2_hi(r2);
-  lsum_e = f2_lo(e2) + f2_hi(e2);
+  const uint64_t e2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+  return f2_lo(e2) + f2_hi(e2);
+}
+
+// x rounded to the 16-bit MMA type and back.
+template <bool BF16>
+__device__ __forceinline__ float round16(float x) {
+  if constexpr (BF16) return __bfloat162float(__float2bfloat16_rn(x));
+  else return __half2float(__float2half_rn(x));
 }
 
 template <int D, bool BF16>
@@ -442,9 +475,11 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
   for (int it = 0; next_unit(p, it, U); ++it) {
     if (U.n[t] == 0) continue;
     const int row = U.mb[t] * BM + r;
-    // l_r: sum of the rounded P (normalises O, matching what P·V consumed);
-    // l_e: sum of the unrounded P (gives LSE).
-    float m = -INFINITY, l_r = 0.f, l_e = 0.f;
+    // l_e: sum of the unrounded P (gives LSE). l_o normalises O: l_e plus,
+    // per K/V tile, the rounding error of that tile's largest P (the weight
+    // that dominates a peaked row), so that O divides the P·V sum by a
+    // denominator built from the same 16-bit weights where it matters.
+    float m = -INFINITY, l_o = 0.f, l_e = 0.f;
     for (int j = 0; j < U.n[t]; ++j) {
       if (!wait_bar_warp(bar_addr<D>(sbase, BAR_SFULL + t), sf_ph, c)) return;
       sf_ph ^= 1;
@@ -475,12 +510,13 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
       }
       m = m_new;
       const float mref = (m == -INFINITY) ? 0.f : m;
-      float lsum_r, lsum_e;
-      if (masked) exp_store<BF16, true>(s, sl2, mref, t_s, lsum_r, lsum_e);
-      else exp_store<BF16, false>(s, sl2, mref, t_s, lsum_r, lsum_e);
+      const float pmax = ex2_approx(m_cand - mref);  // this tile's largest P
+      const float delta = round16<BF16>(pmax) - pmax;
+      const float lsum = masked ? exp_store<BF16, true>(s, sl2, mref, t_s)
+                                : exp_store<BF16, false>(s, sl2, mref, t_s);
       tmem_wait_st();
-      l_r = l_r * alpha + lsum_r;
-      l_e = l_e * alpha + lsum_e;
+      l_e = l_e * alpha + lsum;
+      l_o = l_o * alpha + (lsum + delta);
       tc_fence_before();
       mbar_arrive(bar_addr<D>(sbase, BAR_PFULL + t));
     }
@@ -488,7 +524,7 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
     // the epilogue of unit k has read it (the next-but-one unit's first P·V
     // waits for that epilogue to free O), so no barrier runs a phase ahead.
     const int buf = units_done & 1;
-    stats[(buf * 2 + t) * BM + r] = make_float4(m, l_r, l_e, 0.f);
+    stats[(buf * 2 + t) * BM + r] = make_float4(m, l_o, l_e, 0.f);
     ++units_done;
     mbar_arrive(bar_addr<D>(sbase, BAR_STATS + 2 * t + buf));
   }
@@ -704,6 +740,22 @@ __global__ void fa_wait_selftest_kernel(unsigned long long timeout_ns, int* out)
     const bool ok = wait_bar(smem_addr(&bar), 0, c);
     out[0] = ok ? 1 : 0;
     out[1] = abort_flag;
+  }
+}
+
+// Evaluates the FMA-pipe exponential and ex2.approx on n inputs.
+__global__ void fa_exp2_selftest_kernel(const float* x, float* y_fma, float* y_mufu, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const uint64_t e = exp2_fma2(f2_pack(x[i], x[i + 1]));
+    y_fma[i] = f2_lo(e);
+    y_fma[i + 1] = f2_hi(e);
+    y_mufu[i] = ex2_approx(x[i]);
+    y_mufu[i + 1] = ex2_approx(x[i + 1]);
+  } else if (i < n) {
+    const uint64_t e = exp2_fma2(f2_pack(x[i], 0.f));
+    y_fma[i] = f2_lo(e);
+    y_mufu[i] = ex2_approx(x[i]);
   }
 }
 
@@ -960,6 +1012,19 @@ int fa_get_device_status(void) {
   if (cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(int)) != cudaSuccess)
     return fail(FA_ERR_CUDA, "clearing the status word failed");
   return status;
+}
+
+int fa_selftest_exp2(const float* x, float* y_fma, float* y_mufu, int n) {
+  if (n < 1) return fail(FA_ERR_INVALID_ARG, "n must be >= 1");
+  int rc;
+  if ((rc = check_range("x", x, (size_t)n * 4, 4)) != FA_OK) return rc;
+  if ((rc = check_range("y_fma", y_fma, (size_t)n * 4, 4)) != FA_OK) return rc;
+  if ((rc = check_range("y_mufu", y_mufu, (size_t)n * 4, 4)) != FA_OK) return rc;
+  const int pairs = (n + 1) / 2;
+  fa::fa_exp2_selftest_kernel<<<(pairs + 255) / 256, 256>>>(x, y_fma, y_mufu, n);
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "exp2 self test: %s", cudaGetErrorString(e));
+  return FA_OK;
 }
 
 // Runs the bounded wait on a barrier that nothing arrives at, with a limit of

@@ -188,6 +188,23 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+// acc + (lo half of h) + (hi half of h), the halves read as bf16 (BF16) or
+// fp16, accumulated in fp32 (sm_100 mixed-precision add: no unpacking).
+template <bool BF16>
+__device__ __forceinline__ float add_f32_x16x2(float acc, uint32_t h) {
+  float d;
+  if constexpr (BF16) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %1;\n\tadd.rn.f32.bf16 %0, hi, %0;\n\t}"
+        : "=f"(d) : "f"(acc), "r"(h));
+  } else {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.f16 %0, lo, %1;\n\tadd.rn.f32.f16 %0, hi, %0;\n\t}"
+        : "=f"(d) : "f"(acc), "r"(h));
+  }
+  return d;
+}
+
 // Three-input max/min (sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
