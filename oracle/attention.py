@@ -21,8 +21,8 @@ What it computes, and where the pages say so (page title, then section):
 * [CSDN] aicoding.csdn.net page on ops-transformer FlashAttention, "第一层，
   算子融合": the mask is applied inside the fused kernel.
 
-Readings taken where the pages are silent or garbled (each is listed in
-the design doc): the mask is additive −inf after scaling; causal allows key j when
+Readings taken where the pages are silent or garbled: the mask is additive
+−inf after scaling; causal allows key j when
 j <= i; key padding removes keys j >= L_b and still computes every query row;
 LSE_i = ln Σ_j exp(scale·q_i·k_j) over allowed j; query head hq reads K/V head
 hq // (Hq / Hk); a row with no allowed key has O = 0 and LSE = −inf.

@@ -383,7 +383,7 @@ __device__ __forceinline__ uint64_t exp2_fma2(uint64_t y) {
   return ((uint64_t)r1 << 32) | r0;
 }
 // One pair in every EXP2_FMA_EVERY takes the FMA-pipe exponential (unmasked tiles).
-constexpr int EXP2_FMA_EVERY = 1 << 30;  // off: measured slower here
+constexpr int EXP2_FMA_EVERY = 1 << 30;  // off: slower than ex2.approx alone in this kernel
 
 // Row max of one S tile for this thread's row, in log2 units of the scaled
 // score. MASKED: keys c >= nvalid are masked, and s is rewritten in place to
