@@ -247,6 +247,27 @@ def config_of(w, n):
                   "L2 flushed between steps (256 MB write)"}
 
 
+def rank_inputs(w, rank):
+    """This rank's independent shard of the workload: the same shapes with a
+    seed shifted by the rank (no data is exchanged between ranks)."""
+    return make_inputs(w, batch_offset=rank)
+
+
+def max_over_ranks(x, world, device="cpu"):
+    """Slowest rank's value (the whole job ends when the last rank does)."""
+    if world == 1:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flop_per_rank, world, ms_per_step):
+    """Aggregate throughput: the FLOP of every rank's step over the slowest step time."""
+    return flop_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def in_bytes(w):
     return 2 * w.B * w.N * w.d * (w.Hq + 2 * w.Hk)
 
@@ -286,14 +307,10 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(x):
+        return max_over_ranks(x, world, dev)
 
-    x = make_inputs(w, batch_offset=rank)
+    x = rank_inputs(w, rank)
     q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
     lens = x["key_pad_lens"].to(dev) if x["key_pad_lens"] is not None else None
     o = torch.empty_like(q)
@@ -334,9 +351,9 @@ def main():
         torch.cuda.synchronize()
         barrier()
     status = binding.device_status()
-    total_ms = max_over_ranks(t_begin.elapsed_time(t_end))
+    total_ms = rank_max(t_begin.elapsed_time(t_end))
     kern_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    kern_avg = max_over_ranks(sum(kern_ms) / len(kern_ms))
+    kern_avg = rank_max(sum(kern_ms) / len(kern_ms))
 
     # ---- end-to-end through the public API: pinned host inputs in, O and LSE out
     hq_, hk_, hv_ = (x[n].pin_memory() for n in ("q", "k", "v"))
@@ -366,7 +383,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+    e2e_ms = rank_max(e0.elapsed_time(e1)) / e2e_steps
     h2d = sum(t.numel() * t.element_size() for t in (hq_, hk_, hv_)) + \
         (hlens.numel() * 4 if hlens is not None else 0)
     d2h = ho.numel() * ho.element_size() + hl.numel() * 4
@@ -378,7 +395,7 @@ def main():
 
     f = flops(w)
     ms_per_step = total_ms / args.steps
-    value = f * world / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(f, world, ms_per_step)
     peak, peak_src = peaks()
     achieved = f / (kern_avg * 1e-3) / 1e12
     traffic = recorded_traffic(w.name)
@@ -392,7 +409,7 @@ def main():
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                      "kernel": "fa_fwd_kernel", "kernel_ms": kern_avg,
                      "flop_per_launch": f},
-        "e2e": {"value": f * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": whole_job_tflops(f, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "steps": e2e_steps},
         "gpu_launches": args.steps,
