@@ -71,7 +71,8 @@ enum {
   BAR_OFREE = 14,   // [2] epilogue -> MMA: O read out of TMEM
   BAR_STATS = 16,   // [2 tiles][2 buffers] softmax -> epilogue: final m, l in smem
   BAR_DRAIN = 20,   // MMA drain on the abort path
-  BAR_KV = 21       // [STAGES] full, then [STAGES] empty
+  BAR_PHALF = 21,   // [2] softmax -> MMA: P of the first 64 keys written to TMEM
+  BAR_KV = 23       // [STAGES] full, then [STAGES] empty
 };
 
 template <int D>
@@ -124,7 +125,9 @@ struct Ctl {
 __device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, const Ctl& c) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    // Sleep in the barrier (up to 0.2 ms per try) rather than spin: waiting
+    // warps share issue slots with the softmax warps on the same SMSP.
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
     if (*c.abort_flag) return false;
     if (global_timer_ns() - t0 > c.timeout_ns) {
       *c.abort_flag = 1;
@@ -251,20 +254,22 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
       umma_ss_warp(d_s, qd + off, kd + off, IDESC_QK, 1u);
     }
   };
-  auto issue_pv = [&](int t, int vst, uint32_t acc) {
+  // P·V over keys [32·h, 32·h + 64) of the tile (h = 0: first half, 1: second).
+  auto issue_pv_half = [&](int t, int vst, int h, uint32_t acc) {
     // P: 16 keys = 8 TMEM columns (two 16-bit values per column); V: 16 key
     // rows of 128 bytes in each 64-column box, boxes SW128_BOX_BYTES apart.
     const uint64_t vd = v_desc0 + (uint64_t)((vst * L::KV_BYTES) >> 4);
     const uint32_t d_o = tmem + TmemO<D>::col(t);
     const uint32_t a_p = tmem + S_COL[t];
-    umma_ts_warp(d_o, a_p, vd, IDESC_PV, acc);
+    const int k0 = h * (BN / 32);
+    umma_ts_warp(d_o, a_p + k0 * 8, vd + ((k0 * 16 * 128) >> 4), IDESC_PV, acc);
 #pragma unroll
-    for (int k = 1; k < BN / 16; ++k)
+    for (int k = k0 + 1; k < k0 + BN / 32; ++k)
       umma_ts_warp(d_o, a_p + k * 8, vd + ((k * 16 * 128) >> 4), IDESC_PV, 1u);
   };
 
   // Phase bits, one per barrier the MMA thread waits on.
-  constexpr uint32_t QF = 0, PF = 2, OC = 4, OF = 6;
+  constexpr uint32_t QF = 0, PF = 2, OC = 4, OF = 6, PH = 8;
   uint32_t ph = 0;
   auto wait_flip = [&](int bar, uint32_t bit, uint32_t invert) {
     const bool r = wait_bar_warp(bar_addr<D>(sbase, bar), ((ph >> bit) & 1u) ^ invert, c);
@@ -308,14 +313,17 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
       for (int t = 0; t < 2; ++t) {
         const int nt = t ? n1 : n0;
         if (j >= nt) continue;
-        if (!(ok = wait_flip(BAR_PFULL + t, PF + t, 0))) break;
+        if (!(ok = wait_flip(BAR_PHALF + t, PH + t, 0))) break;
         if (j > 0) {
           if (!(ok = wait_flip(BAR_OCORR + t, OC + t, 0))) break;
         } else {
           if (!(ok = wait_flip(BAR_OFREE + t, OF + t, 1))) break;
         }
         tc_fence_after();
-        issue_pv(t, vs, j > 0 ? 1u : 0u);
+        issue_pv_half(t, vs, 0, j > 0 ? 1u : 0u);
+        if (!(ok = wait_flip(BAR_PFULL + t, PF + t, 0))) break;
+        tc_fence_after();
+        issue_pv_half(t, vs, 1, 1u);
         if (j == nt - 1) {
           umma_commit_warp(bar_addr<D>(sbase, BAR_PVDONE + t));
           umma_commit_warp(bar_addr<D>(sbase, BAR_QEMPTY + t));
@@ -421,12 +429,12 @@ __device__ __forceinline__ float row_max(uint32_t (&s)[BN], float sl2, int nvali
 }
 
 // P = exp2(s·scale·log2e − mref) for this thread's row, rounded to 16 bits and
-// written over S in TMEM; returns the sum of the unrounded P. The whole row is
-// computed before the two TMEM stores so that the exponentials of all 128
-// columns can overlap; scale-and-subtract and the sum use packed fp32 pairs.
+// written over S in TMEM in two 64-key halves (arriving on half_bar after the
+// first); returns the sum of the unrounded P. Scale-and-subtract and the sum
+// use packed fp32 pairs.
 template <bool BF16, bool MASKED>
 __device__ __forceinline__ float exp_store(const uint32_t (&s)[BN], float sl2, float mref,
-                                           uint32_t t_p) {
+                                           uint32_t t_p, uint32_t half_bar) {
   const uint64_t k2 = f2_pack(sl2, sl2), nm2 = f2_pack(-mref, -mref);
   uint64_t acc[4] = {0, 0, 0, 0};
   uint32_t pk[BN / 2];
@@ -445,8 +453,15 @@ __device__ __forceinline__ float exp_store(const uint32_t (&s)[BN], float sl2, f
     }
     acc[i & 3] = fadd2(acc[i & 3], f2_pack(p0, p1));
     pk[i] = round_pack<BF16>(p0, p1);
+    if (i == BN / 4 - 1) {
+      // First 64 keys: store and signal now, so the P·V MMA on them can
+      // overlap the second half of the exponentials.
+      tmem_st_x32(t_p, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(half_bar);
+    }
   }
-  tmem_st_x32(t_p, pk);
   tmem_st_x32(t_p + 32, pk + 32);
   const uint64_t e2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
   return f2_lo(e2) + f2_hi(e2);
@@ -512,8 +527,9 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
       const float mref = (m == -INFINITY) ? 0.f : m;
       const float pmax = ex2_approx(m_cand - mref);  // this tile's largest P
       const float delta = round16<BF16>(pmax) - pmax;
-      const float lsum = masked ? exp_store<BF16, true>(s, sl2, mref, t_s)
-                                : exp_store<BF16, false>(s, sl2, mref, t_s);
+      const uint32_t half_bar = bar_addr<D>(sbase, BAR_PHALF + t);
+      const float lsum = masked ? exp_store<BF16, true>(s, sl2, mref, t_s, half_bar)
+                                : exp_store<BF16, false>(s, sl2, mref, t_s, half_bar);
       tmem_wait_st();
       l_e = l_e * alpha + lsum;
       l_o = l_o * alpha + (lsum + delta);
@@ -672,6 +688,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bar_addr<D>(sbase, BAR_QEMPTY + t), 1);
       mbar_init(bar_addr<D>(sbase, BAR_SFULL + t), 1);
       mbar_init(bar_addr<D>(sbase, BAR_PFULL + t), BM);
+      mbar_init(bar_addr<D>(sbase, BAR_PHALF + t), BM);
       mbar_init(bar_addr<D>(sbase, BAR_AFULL + t), BM);
       mbar_init(bar_addr<D>(sbase, BAR_OCORR + t), BM);
       mbar_init(bar_addr<D>(sbase, BAR_PVDONE + t), 1);
