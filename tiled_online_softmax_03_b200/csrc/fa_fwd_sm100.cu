@@ -62,7 +62,7 @@ struct TmemO {
 // Barrier slots.
 enum {
   BAR_QFULL = 0,    // [2] TMA -> MMA: Q tile loaded
-  BAR_QEMPTY = 2,   // [2] MMA -> TMA: all QK of the unit done with Q tile
+  BAR_QEMPTY = 2,   // [2] MMA -> TMA: the unit's last QK no longer needs the Q tile
   BAR_SFULL = 4,    // [2] MMA -> softmax: S tile ready in TMEM
   BAR_PFULL = 6,    // [2] softmax -> MMA: P written to TMEM
   BAR_AFULL = 8,    // [2] softmax -> correction: rescale factors in smem
@@ -287,13 +287,17 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
     if (n0 > 0 && !(ok = wait_flip(BAR_QFULL + 0, QF + 0, 0))) break;
     if (n1 > 0 && !(ok = wait_flip(BAR_QFULL + 1, QF + 1, 0))) break;
     tc_fence_after();
+    // Q_t is released (QEMPTY) as soon as the unit's last S_t MMA is issued,
+    // so the next unit's Q tile loads while this unit's softmax and P·V run.
     if (n0 > 0) {
       issue_qk(0, k0);
       umma_commit_warp(bar_addr<D>(sbase, BAR_SFULL + 0));
+      if (n0 == 1) umma_commit_warp(bar_addr<D>(sbase, BAR_QEMPTY + 0));
     }
     if (n1 > 0) {
       issue_qk(1, k0);
       umma_commit_warp(bar_addr<D>(sbase, BAR_SFULL + 1));
+      if (n1 == 1) umma_commit_warp(bar_addr<D>(sbase, BAR_QEMPTY + 1));
     }
     umma_commit_warp(bar_addr<D>(sbase, BAR_KV + L::STAGES + k0));
 
@@ -326,7 +330,6 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
         issue_pv_half(t, vs, 1, 1u);
         if (j == nt - 1) {
           umma_commit_warp(bar_addr<D>(sbase, BAR_PVDONE + t));
-          umma_commit_warp(bar_addr<D>(sbase, BAR_QEMPTY + t));
         } else {
           if (!kn_ready) {
             if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_KV + kn), kn_ph, c))) break;
@@ -335,6 +338,7 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
           }
           issue_qk(t, kn);
           umma_commit_warp(bar_addr<D>(sbase, BAR_SFULL + t));
+          if (j + 2 == nt) umma_commit_warp(bar_addr<D>(sbase, BAR_QEMPTY + t));
         }
       }
       if (!ok) break;
@@ -617,8 +621,8 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
         pv_ph[t] ^= 1;
         tc_fence_after();
         if (ml.y > 0.f) {
-          inv_l = 1.f / ml.y;
-          lse = (ml.x + log2f(ml.z)) * 0.69314718055994531f;
+          inv_l = __frcp_rn(ml.y);
+          lse = (ml.x + __log2f(ml.z)) * 0.69314718055994531f;
         }
       }
       const int slab_row0 = U.mb[t] * BM + 32 * wl;
