@@ -20,6 +20,11 @@ What it computes, and where the pages say so (page title, then section):
   "坑四" (GQA/MQA: K and V carry fewer heads than Q).
 * [CSDN] aicoding.csdn.net page on ops-transformer FlashAttention, "第一层，
   算子融合": the mask is applied inside the fused kernel.
+* [GQA] "深度探索Flash-Attention中GQA性能调优技术解析", section
+  "num_splits参数的场景化配置": the attention work of one problem may be cut
+  into num_splits parts. Read here as a split of the key range, each part's
+  result merged by its log-sum-exp (the section gives no formula; the merge is
+  the [MCU] §二 recurrence with a whole key range as one tile).
 
 Readings taken where the pages are silent or garbled: the mask is additive
 −inf after scaling; causal allows key j when
@@ -41,6 +46,9 @@ __all__ = [
     "attention_rows",
     "online_attention_flowchart",
     "online_attention_equations",
+    "attention_key_range",
+    "merge_splits",
+    "split_kv_attention",
 ]
 
 
@@ -244,3 +252,64 @@ def online_attention_equations(q, k, v, scale, causal=False, key_pad_lens=None,
     """Tiled attention with the online recurrence of [MCU] §二 (equation form)."""
     return _online(q, k, v, scale, causal, key_pad_lens, tile_r, tile_c,
                    _update_equations)
+
+
+def attention_key_range(q, k, v, scale, causal, key_pad_lens, key_lo, key_hi):
+    """Attention with only keys key_lo <= j < key_hi allowed (one part of [GQA]'s split).
+
+    The same definition as `attention`, with the key range as one more mask
+    term. Returns (O_s, LSE_s): O_s is normalised by this range's own
+    denominator; a row with no allowed key in the range has O_s = 0 and
+    LSE_s = −inf.
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, Hq, N, _ = q.shape
+    group = Hq // k.shape[1]
+    o = np.zeros((B, Hq, N, v.shape[3]), dtype=np.float64)
+    lse = np.full((B, Hq, N), -np.inf, dtype=np.float64)
+    j = np.arange(N)[None, :]
+    in_range = (j >= key_lo) & (j < key_hi)
+    for b in range(B):
+        key_len = _key_len(key_pad_lens, b, N)
+        for hq in range(Hq):
+            hk = hq // group
+            rows = np.arange(N)
+            ok = allowed_keys(rows, N, causal, key_len) & in_range
+            s = scores(q[b, hq], k[b, hk], scale, ok)
+            p, m, l = two_pass_softmax(s)
+            o[b, hq], lse[b, hq] = _finish(p, m, l, v[b, hk])
+    return o, lse
+
+
+def merge_splits(o_parts, lse_parts):
+    """Result over the union of disjoint key ranges from each range's (O_s, LSE_s).
+
+    With m = max_s LSE_s and w_s = exp(LSE_s − m) (0 for LSE_s = −inf):
+    O = Σ_s w_s O_s / Σ_s w_s and LSE = m + ln Σ_s w_s. Since LSE_s = m_s +
+    ln l_s, w_s is l_s·exp(m_s − m): the [MCU] §二 update of m, l and the
+    unnormalised O with one range as the tile. Rows with no allowed key in
+    any range get O = 0 and LSE = −inf.
+    """
+    o_parts = [_as_f64(x) for x in o_parts]
+    lse_parts = [_as_f64(x) for x in lse_parts]
+    m = np.max(np.stack(lse_parts), axis=0)
+    has = np.isfinite(m)
+    m_safe = np.where(has, m, 0.0)
+    num = np.zeros(o_parts[0].shape)
+    den = np.zeros(m.shape)
+    for o_s, lse_s in zip(o_parts, lse_parts):
+        w = np.where(np.isfinite(lse_s), np.exp(np.where(np.isfinite(lse_s), lse_s, 0.0) - m_safe), 0.0)
+        num += w[..., None] * o_s
+        den += w
+    o = np.zeros(num.shape)
+    o[has] = num[has] / den[has][..., None]
+    lse = np.full(m.shape, -np.inf)
+    lse[has] = m[has] + np.log(den[has])
+    return o, lse
+
+
+def split_kv_attention(q, k, v, scale, causal, key_pad_lens, bounds):
+    """[GQA]'s split: keys cut at `bounds` (0 = c_0 < c_1 < ... = N), merged by LSE."""
+    parts = [attention_key_range(q, k, v, scale, causal, key_pad_lens, lo, hi)
+             for lo, hi in zip(bounds[:-1], bounds[1:])]
+    return merge_splits([p[0] for p in parts], [p[1] for p in parts])

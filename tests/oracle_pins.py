@@ -23,8 +23,10 @@ def rand(*shape, rng=RNG):
     return rng.standard_normal(shape)
 
 
-def brute_force(q, k, v, scale, causal, lens):
-    """Scalar loops with math.fsum: one row at a time, no vectorised code."""
+def brute_force(q, k, v, scale, causal, lens, key_lo=0, key_hi=None):
+    """Scalar loops with math.fsum: one row at a time, no vectorised code.
+
+    Only keys key_lo <= j < key_hi take part (all keys by default)."""
     B, Hq, N, d = q.shape
     Hk = k.shape[1]
     G = Hq // Hk
@@ -35,7 +37,8 @@ def brute_force(q, k, v, scale, causal, lens):
         for h in range(Hq):
             kh = h // G
             for i in range(N):
-                keys = [j for j in range(N) if j < L and (not causal or j <= i)]
+                hi = N if key_hi is None else key_hi
+                keys = [j for j in range(key_lo, hi) if j < L and (not causal or j <= i)]
                 if not keys:
                     continue
                 s = {j: scale * math.fsum(q[b, h, i, c] * k[b, kh, j, c] for c in range(d))
@@ -345,6 +348,56 @@ def load_golden(name="hand_worked.json"):
         out.append({key: (np.array(_golden_value(c[key]), dtype=np.float64)
                           if key in ("q", "k", "v", "o", "lse") else c[key]) for key in c})
     return out
+
+
+# ------------------------------------------------ split-KV ([GQA] num_splits)
+
+def pin_key_range_matches_scalar_brute_force(orc):
+    q, k, v = rand(1, 2, 7, 3), rand(1, 1, 7, 3), rand(1, 1, 7, 2)
+    for causal, lens, lo, hi in itertools.product([False, True], [None, [5]], [0, 2, 3], [3, 6, 7]):
+        o, lse = orc.attention_key_range(q, k, v, 0.9, causal, lens, lo, hi)
+        ob, lseb = brute_force(q, k, v, 0.9, causal, lens, lo, hi)
+        close(o, ob)
+        close(lse, lseb)
+
+
+def pin_split_kv_equals_attention_for_every_cut(orc):
+    """Every way of cutting 6 keys into ranges merges back to the full result."""
+    rng = np.random.default_rng(11)
+    N = 6
+    q, k, v = rng.standard_normal((2, 2, N, 3)), rng.standard_normal((2, 1, N, 3)), \
+        rng.standard_normal((2, 1, N, 2))
+    for causal, lens in [(False, None), (True, None), (False, [4, 0]), (True, [2, 6])]:
+        ref_o, ref_l = orc.attention(q, k, v, 1.1, causal, lens)
+        for mask in range(1 << (N - 1)):
+            cuts = [c for c in range(1, N) if mask >> (c - 1) & 1]
+            o, l = orc.split_kv_attention(q, k, v, 1.1, causal, lens, [0] + cuts + [N])
+            close(o, ref_o, 1e-12)
+            close(l, ref_l, 1e-12)
+
+
+def pin_merge_closed_form(orc):
+    """Two ranges with denominators 1 and 3 at the same max: weights 1/4, 3/4."""
+    a, b = np.array([[2.0, -1.0]]), np.array([[6.0, 3.0]])
+    o, lse = orc.merge_splits([a, b], [np.array([0.0]), np.array([math.log(3.0)])])
+    close(o, [[5.0, 2.0]], 1e-15)
+    close(lse, [math.log(4.0)], 1e-15)
+    # a range with no allowed key (LSE −inf) has weight 0; no range at all gives 0 / −inf
+    o, lse = orc.merge_splits([a, b, b], [np.array([-math.inf]), np.array([1.5]), np.array([-math.inf])])
+    close(o, b, 1e-15)
+    close(lse, [1.5], 1e-15)
+    o, lse = orc.merge_splits([a, b], [np.array([-math.inf]), np.array([-math.inf])])
+    close(o, [[0.0, 0.0]])
+    close(lse, [-math.inf])
+
+
+def pin_merge_large_lse_stays_finite(orc):
+    """LSE 800 and 799 overflow exp() unless the max is taken out first."""
+    a, b = np.array([[1.0]]), np.array([[0.0]])
+    o, lse = orc.merge_splits([a, b], [np.array([800.0]), np.array([799.0])])
+    e = math.e
+    close(o, [[e / (e + 1.0)]], 1e-14)
+    close(lse, [800.0 + math.log1p(1.0 / e)], 1e-15)
 
 
 def pin_hand_worked_golden(orc):

@@ -43,6 +43,15 @@ MUTATIONS = {
     "v_rows_reversed": ("rows] = _finish(p, m, l, v[b, hk])", "rows] = _finish(p, m, l, v[b, hk][::-1])"),
     "k_rows_reversed": ("s = scores(q[b, hq, rows], k[b, hk], scale, ok)",
                         "s = scores(q[b, hq, rows], k[b, hk][::-1], scale, ok)"),
+    "key_range_hi_inclusive": ("in_range = (j >= key_lo) & (j < key_hi)",
+                               "in_range = (j >= key_lo) & (j <= key_hi)"),
+    "key_range_lo_exclusive": ("in_range = (j >= key_lo) & (j < key_hi)",
+                               "in_range = (j > key_lo) & (j < key_hi)"),
+    "merge_max_not_subtracted": ("np.exp(np.where(np.isfinite(lse_s), lse_s, 0.0) - m_safe)",
+                                 "np.exp(np.where(np.isfinite(lse_s), lse_s, 0.0))"),
+    "merge_unweighted": ("num += w[..., None] * o_s", "num += o_s"),
+    "merge_unnormalised": ("o[has] = num[has] / den[has][..., None]", "o[has] = num[has]"),
+    "merge_lse_without_max": ("lse[has] = m[has] + np.log(den[has])", "lse[has] = np.log(den[has])"),
 }
 
 
