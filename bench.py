@@ -281,6 +281,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shape", default=None,
+                    help="B,Hq,Hk,N[,causal] replacing the workload's shape (other settings kept)")
+    ap.add_argument("--splits", type=int, default=1,
+                    help="K/V splits per Q tile pair (fa_fwd_splitkv; 1 = fa_fwd)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -288,6 +292,12 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     w = WORKLOADS[args.workload]
+    if args.shape:
+        f = [int(t) for t in args.shape.split(",")]
+        kw = dict(B=f[0], Hq=f[1], Hk=f[2], N=f[3])
+        if len(f) > 4:
+            kw["causal"] = bool(f[4])
+        w = w.with_(name=f"{w.name}@" + "x".join(str(t) for t in f), key_pad=None, **kw)
 
     if args.impl == "reference":
         run_reference(args, w, rank)
@@ -319,12 +329,24 @@ def main():
     if in_bytes(w) <= 126e6:
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    ws = None
+    if args.splits > 1:
+        ws = torch.empty(binding.splitkv_workspace_bytes(w.B, w.Hq, w.N, w.d, args.splits),
+                         dtype=torch.uint8, device=dev)
+
+    def call():
+        if args.splits > 1:
+            binding.fa_fwd_splitkv(q, k, v, args.splits, causal=w.causal, scale=w.scale,
+                                   key_pad_lens=lens, out=o, lse=lse, workspace=ws,
+                                   stream=stream.cuda_stream)
+        else:
+            binding.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, key_pad_lens=lens, out=o,
+                           lse=lse, stream=stream.cuda_stream)
 
     def step():
         if flush is not None:
             flush.fill_(1)
-        binding.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, key_pad_lens=lens, out=o, lse=lse,
-                       stream=stream.cuda_stream)
+        call()
 
     for _ in range(args.warmup):
         step()
@@ -344,8 +366,7 @@ def main():
             if flush is not None:
                 flush.fill_(1)
             starts[i].record(stream)
-            binding.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, key_pad_lens=lens, out=o,
-                           lse=lse, stream=stream.cuda_stream)
+            call()
             ends[i].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -368,8 +389,7 @@ def main():
         v.copy_(hv_, non_blocking=True)
         if hlens is not None:
             lens.copy_(hlens, non_blocking=True)
-        binding.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, key_pad_lens=lens, out=o, lse=lse,
-                       stream=stream.cuda_stream)
+        call()
         ho.copy_(o, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
 
@@ -398,21 +418,26 @@ def main():
     value = whole_job_tflops(f, world, ms_per_step)
     peak, peak_src = peaks()
     achieved = f / (kern_avg * 1e-3) / 1e12
-    traffic = recorded_traffic(w.name)
+    traffic = recorded_traffic(w.name) if args.splits == 1 else None
+    config = config_of(w, world)
+    kernels = "fa_fwd_kernel"
+    if args.splits > 1:
+        config["num_splits"] = args.splits
+        kernels = "fa_fwd_kernel + fa_merge_splits_kernel"
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
-        "config": config_of(w, world),
+        "config": config,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
-                     "kernel": "fa_fwd_kernel", "kernel_ms": kern_avg,
+                     "kernel": kernels, "kernel_ms": kern_avg,
                      "flop_per_launch": f},
         "e2e": {"value": whole_job_tflops(f, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "steps": e2e_steps},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * (2 if args.splits > 1 else 1),
         "clocks": clocks.summary(),
         "device_status": status,
     }

@@ -41,6 +41,7 @@
 #ifndef FA_H_
 #define FA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -83,6 +84,42 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            int B, int Hq, int Hk, int N, int d, float scale, int causal,
            const int32_t* key_pad_lens, void* stream, int dtype);
 
+/*
+ * Split-KV forward (the num_splits setting of the GQA page "深度探索Flash-
+ * Attention中GQA性能调优技术解析", section "num_splits参数的场景化配置"): the
+ * K/V tiles each pair of Q tiles visits are cut into `num_splits` contiguous
+ * chunks processed by separate work units, so a problem with few Q tiles
+ * still fills the GPU. Each chunk's result (O normalised by its own
+ * denominator and its LSE, fp32) goes to `workspace`; a second kernel on the
+ * same stream merges the chunks row by row by log-sum-exp:
+ *     m = max_s LSE_s,  w_s = exp(LSE_s − m),
+ *     O = Σ_s w_s O_s / Σ_s w_s,  LSE = m + ln Σ_s w_s
+ * (a chunk with no allowed key has LSE_s = −inf and weight 0). The result
+ * equals fa_fwd's up to fp32 rounding.
+ *
+ *   num_splits       1..16. With 1 this is fa_fwd (workspace unused, may be NULL).
+ *   workspace        device pointer, 256-byte aligned, at least
+ *                    fa_splitkv_workspace_bytes(B, Hq, N, d, num_splits) bytes,
+ *                    overlapping no other argument. Owned by the caller; its
+ *                    contents need no initialisation and are scratch after the
+ *                    call. Two calls in flight at once (other streams) need
+ *                    two workspaces.
+ *   workspace_bytes  size of `workspace`.
+ *   other arguments  as for fa_fwd.
+ * Returns as fa_fwd: FA_OK after enqueuing both kernels, or a negative
+ * fa_status (FA_ERR_INVALID_ARG for a bad split count, a short, misaligned or
+ * overlapping workspace) with nothing enqueued.
+ */
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int Hq, int Hk, int N, int d, float scale, int causal,
+                   const int32_t* key_pad_lens, int num_splits, void* workspace,
+                   size_t workspace_bytes, void* stream, int dtype);
+
+/* Workspace bytes fa_fwd_splitkv needs: B·Hq·N·num_splits·(d + 1) floats,
+ * each part rounded up to 256 bytes; 0 for num_splits == 1 and for invalid
+ * arguments. */
+size_t fa_splitkv_workspace_bytes(int B, int Hq, int N, int d, int num_splits);
+
 /* Message for the last error returned to the calling thread ("" if none).
  * The string is owned by the library (thread-local storage). */
 const char* fa_last_error_string(void);
@@ -108,6 +145,13 @@ int fa_num_units(int B, int Hq, int Hk, int N, int causal);
 /* Decodes unit u into out[8] = {b, hk, hq0, mblock0, present0, hq1, mblock1,
  * present1}. Returns FA_OK or FA_ERR_INVALID_ARG. */
 int fa_unit_info(int B, int Hq, int Hk, int N, int causal, int u, int32_t* out);
+
+/* With split-KV: unit u of a `num_splits` launch, for a batch whose valid key
+ * count is key_len, into out[12] = {b, hk, hq0, mblock0, present0, hq1,
+ * mblock1, present1, split, j0, n0, n1}: Q tile t visits K/V tiles
+ * [j0, n_t) (none when n_t <= j0). Returns FA_OK or FA_ERR_INVALID_ARG. */
+int fa_unit_kv_range(int B, int Hq, int Hk, int N, int causal, int num_splits, int u,
+                     int key_len, int32_t* out);
 
 /* Unit taken by CTA `cta` of a `grid`-CTA launch on its iteration `it`
  * (may be >= fa_num_units, meaning that CTA is done). */

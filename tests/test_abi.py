@@ -122,3 +122,57 @@ def test_serpentine_assignment_is_a_partition(grid, units):
 def test_unit_info_rejects_bad_index():
     with pytest.raises(binding.FaError):
         binding.unit_info(1, 1, 1, 128, 0, 5)
+
+
+# ----------------------------------------------------- split-KV decomposition
+
+SPLIT_SHAPES = [(1, 1, 1, 128, 0), (2, 4, 2, 300, 1), (2, 3, 1, 513, 0), (1, 8, 1, 2048, 1),
+                (1, 6, 2, 1000, 1), (3, 5, 5, 129, 1), (1, 2, 2, 1, 0)]
+
+
+def needed_tiles(N, causal, mb, key_len):
+    end = min(key_len, (mb + 1) * 128) if causal else key_len
+    return (end + 127) // 128 if end > 0 else 0
+
+
+@pytest.mark.parametrize("B,Hq,Hk,N,causal", SPLIT_SHAPES)
+@pytest.mark.parametrize("splits", [1, 2, 3, 4, 7, 16])
+def test_split_ranges_partition_each_tiles_keys(B, Hq, Hk, N, causal, splits):
+    """Across the splits of a tile pair, each Q tile visits every K/V tile it
+    needs exactly once, and a split's tiles are one contiguous range."""
+    nu = binding.num_units(B, Hq, Hk, N, causal)
+    for key_len in sorted({N, max(N // 3, 1), 1, 0}):
+        visits = {}
+        for u in range(nu * splits):
+            r = binding.unit_kv_range(B, Hq, Hk, N, causal, splits, u, key_len)
+            assert r[:8] == binding.unit_info(B, Hq, Hk, N, causal, u // splits)
+            assert r[8] == u % splits
+            j0 = r[9]
+            for t, (hq, mb, present, n) in enumerate(((r[2], r[3], r[4], r[10]),
+                                                      (r[5], r[6], r[7], r[11]))):
+                if not present:
+                    continue
+                assert n >= j0
+                visits.setdefault((r[0], hq, mb), []).extend(range(j0, n))
+        assert len(visits) == B * Hq * ((N + 127) // 128)
+        for (b, hq, mb), tiles in visits.items():
+            assert sorted(tiles) == list(range(needed_tiles(N, causal, mb, key_len)))
+
+
+def test_split_count_and_workspace_size():
+    assert binding.splitkv_workspace_bytes(2, 3, 100, 128, 1) == 0
+    assert binding.splitkv_workspace_bytes(2, 3, 100, 128, 17) == 0
+    assert binding.splitkv_workspace_bytes(2, 3, 100, 96, 2) == 0
+    rows = 2 * 3 * 100 * 4
+    rup = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert binding.splitkv_workspace_bytes(2, 3, 100, 128, 4) == rup(rows * 128 * 4) + rup(rows * 4)
+    assert binding.splitkv_workspace_bytes(1, 1, 1, 64, 16) == 16 * 64 * 4 + 256
+    lib = binding.lib
+    for splits in (0, 17, -1):
+        assert lib.fa_fwd_splitkv(16, 16, 16, 16, None, 1, 1, 1, 128, 64, 0.1, 0, None, splits,
+                                  None, 0, None, 0) == -1
+        assert "num_splits" in binding.last_error()
+    with pytest.raises(binding.FaError):
+        binding.unit_kv_range(1, 1, 1, 128, 0, 2, 2, 128)  # only units 0 and 1 exist
+    with pytest.raises(binding.FaError):
+        binding.unit_kv_range(1, 1, 1, 128, 0, 2, 0, 129)  # key_len > N

@@ -2,7 +2,8 @@
 
 Every step of the attention forward runs in the library's CUDA kernel; this
 module checks tensor metadata, allocates the outputs with torch when the
-caller does not pass them, and calls ``fa_fwd`` on the current torch stream.
+caller does not pass them, and calls ``fa_fwd`` (or ``fa_fwd_splitkv``) on the
+current torch stream.
 Importing it loads the library and raises if it is missing: there is no
 fallback path.
 """
@@ -12,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["FaError", "fa_fwd", "load_library", "lib", "FA_OK", "FA_ERR_INVALID_ARG",
+__all__ = ["FaError", "fa_fwd", "fa_fwd_splitkv", "splitkv_workspace_bytes", "load_library", "lib", "FA_OK", "FA_ERR_INVALID_ARG",
            "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT"]
 
 FA_OK = 0
@@ -42,6 +43,14 @@ def load_library(path=LIB_PATH):
     L.fa_fwd.argtypes = [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                          c_int, c_int, c_float, c_int, c_void_p, c_void_p, c_int]
     L.fa_fwd.restype = c_int
+    L.fa_fwd_splitkv.argtypes = [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int,
+                                 c_int, c_int, c_int, c_float, c_int, c_void_p, c_int, c_void_p,
+                                 ctypes.c_size_t, c_void_p, c_int]
+    L.fa_fwd_splitkv.restype = c_int
+    L.fa_splitkv_workspace_bytes.argtypes = [c_int] * 5
+    L.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
+    L.fa_unit_kv_range.argtypes = [c_int] * 8 + [ctypes.POINTER(ctypes.c_int32)]
+    L.fa_unit_kv_range.restype = c_int
     L.fa_last_error_string.argtypes = []
     L.fa_last_error_string.restype = ctypes.c_char_p
     L.fa_get_device_status.argtypes = []
@@ -77,14 +86,7 @@ def check(code):
 _DTYPES = {torch.float16: FA_FP16, torch.bfloat16: FA_BF16}
 
 
-def fa_fwd(q, k, v, causal=False, scale=None, key_pad_lens=None, out=None, lse=None,
-           return_lse=True, stream=None):
-    """O (and LSE) = attention forward of q [B,Hq,N,d] against k, v [B,Hk,N,d].
-
-    Tensors must be CUDA, contiguous, fp16 or bf16 (all the same). ``scale``
-    defaults to 1/sqrt(d). ``key_pad_lens`` is an int32 CUDA tensor [B] or
-    None. ``out``/``lse`` may be given preallocated. Returns (o, lse) or o.
-    """
+def _prepare(q, k, v, key_pad_lens, out, lse, return_lse, scale, stream):
     for name, t in (("q", q), ("k", k), ("v", v)):
         if not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
             raise FaError(FA_ERR_INVALID_ARG, f"{name} must be a contiguous 4-D CUDA tensor")
@@ -106,12 +108,58 @@ def fa_fwd(q, k, v, causal=False, scale=None, key_pad_lens=None, out=None, lse=N
         scale = float(d) ** -0.5
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
+    return (B, Hq, Hk, N, d), out, lse, float(scale), stream
+
+
+def fa_fwd(q, k, v, causal=False, scale=None, key_pad_lens=None, out=None, lse=None,
+           return_lse=True, stream=None):
+    """O (and LSE) = attention forward of q [B,Hq,N,d] against k, v [B,Hk,N,d].
+
+    Tensors must be CUDA, contiguous, fp16 or bf16 (all the same). ``scale``
+    defaults to 1/sqrt(d). ``key_pad_lens`` is an int32 CUDA tensor [B] or
+    None. ``out``/``lse`` may be given preallocated. Returns (o, lse) or o.
+    """
+    (B, Hq, Hk, N, d), out, lse, scale, stream = _prepare(q, k, v, key_pad_lens, out, lse,
+                                                          return_lse, scale, stream)
     with torch.cuda.device(q.device):
         check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                          lse.data_ptr() if lse is not None else None, B, Hq, Hk, N, d,
-                         float(scale), 1 if causal else 0,
+                         scale, 1 if causal else 0,
                          key_pad_lens.data_ptr() if key_pad_lens is not None else None,
                          stream, _DTYPES[q.dtype]))
+    return (out, lse) if return_lse else out
+
+
+def splitkv_workspace_bytes(B, Hq, N, d, num_splits):
+    """Bytes of scratch ``fa_fwd_splitkv`` needs (0 for one split)."""
+    return lib.fa_splitkv_workspace_bytes(B, Hq, N, d, num_splits)
+
+
+def fa_fwd_splitkv(q, k, v, num_splits, causal=False, scale=None, key_pad_lens=None, out=None,
+                   lse=None, return_lse=True, workspace=None, stream=None):
+    """As ``fa_fwd``, with each Q tile pair's K/V range cut into ``num_splits``
+    chunks (1..16) whose partial results a second kernel merges by LSE.
+
+    ``workspace`` is a CUDA tensor of at least ``splitkv_workspace_bytes``
+    bytes (allocated here when None); a call in flight owns it until the
+    stream reaches the end of the merge.
+    """
+    (B, Hq, Hk, N, d), out, lse, scale, stream = _prepare(q, k, v, key_pad_lens, out, lse,
+                                                          return_lse, scale, stream)
+    need = splitkv_workspace_bytes(B, Hq, N, d, num_splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is not None and (not workspace.is_cuda or not workspace.is_contiguous()):
+        raise FaError(FA_ERR_INVALID_ARG, "workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    with torch.cuda.device(q.device):
+        check(lib.fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr() if lse is not None else None, B, Hq, Hk, N, d,
+                                 scale, 1 if causal else 0,
+                                 key_pad_lens.data_ptr() if key_pad_lens is not None else None,
+                                 int(num_splits),
+                                 workspace.data_ptr() if workspace is not None else None,
+                                 ws_bytes, stream, _DTYPES[q.dtype]))
     return (out, lse) if return_lse else out
 
 
@@ -132,3 +180,10 @@ def unit_info(B, Hq, Hk, N, causal, u):
 
 def unit_for(cta, it, grid):
     return lib.fa_unit_for(cta, it, grid)
+
+
+def unit_kv_range(B, Hq, Hk, N, causal, num_splits, u, key_len):
+    """{b, hk, hq0, mb0, present0, hq1, mb1, present1, split, j0, n0, n1} of unit u."""
+    out = (ctypes.c_int32 * 12)()
+    check(lib.fa_unit_kv_range(B, Hq, Hk, N, 1 if causal else 0, num_splits, u, key_len, out))
+    return list(out)

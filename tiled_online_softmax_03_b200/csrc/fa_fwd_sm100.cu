@@ -97,6 +97,8 @@ struct Layout {
 struct Params {
   const int32_t* key_pad_lens;
   float* lse;
+  float* o_part;    // split-KV: [splits][B·Hq][N][d] fp32 partial O (normalised), else null
+  float* lse_part;  // split-KV: [splits][B·Hq][N] fp32 partial LSE
   Shape s;
   float scale_log2;
   unsigned long long timeout_ns;
@@ -179,7 +181,7 @@ __device__ void role_load(const Params& p, uint32_t sbase, const Ctl& c, const C
   Unit U;
   for (int it = 0; ok && next_unit(p, it, U); ++it) {
     for (int t = 0; t < 2 && ok; ++t) {
-      if (U.n[t] == 0) continue;
+      if (!tile_active(U, t)) continue;
       if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_QEMPTY + t), qe_ph[t] ^ 1, c))) break;
       qe_ph[t] ^= 1;
       const uint32_t full = bar_addr<D>(sbase, BAR_QFULL + t);
@@ -192,7 +194,7 @@ __device__ void role_load(const Params& p, uint32_t sbase, const Ctl& c, const C
                     U.mb[t] * BM, head, full);
     }
     const int kv_head = U.b * p.s.Hk + U.hk;
-    for (int j = 0; j < U.nmax && ok; ++j) {
+    for (int j = U.j0; j < U.nmax && ok; ++j) {
       for (int which = 0; which < 2; ++which) {  // K_j then V_j
         if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_KV + L::STAGES + st), kv_ph ^ 1, c))) break;
         const uint32_t full = bar_addr<D>(sbase, BAR_KV + st);
@@ -278,30 +280,30 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
   };
   Unit U;
   for (int it = 0; ok && next_unit(p, it, U); ++it) {
-    const int n0 = U.n[0], n1 = U.n[1], nmax = U.nmax;
-    if (nmax == 0) continue;
+    const int j0 = U.j0, n0 = U.n[0], n1 = U.n[1], nmax = U.nmax;
+    if (nmax == j0) continue;
     const int k0 = st;
     const uint32_t k0_ph = kv_ph;
     if (++st == L::STAGES) { st = 0; kv_ph ^= 1; }
     if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_KV + k0), k0_ph, c))) break;
-    if (n0 > 0 && !(ok = wait_flip(BAR_QFULL + 0, QF + 0, 0))) break;
-    if (n1 > 0 && !(ok = wait_flip(BAR_QFULL + 1, QF + 1, 0))) break;
+    if (n0 > j0 && !(ok = wait_flip(BAR_QFULL + 0, QF + 0, 0))) break;
+    if (n1 > j0 && !(ok = wait_flip(BAR_QFULL + 1, QF + 1, 0))) break;
     tc_fence_after();
     // Q_t is released (QEMPTY) as soon as the unit's last S_t MMA is issued,
     // so the next unit's Q tile loads while this unit's softmax and P·V run.
-    if (n0 > 0) {
+    if (n0 > j0) {
       issue_qk(0, k0);
       umma_commit_warp(bar_addr<D>(sbase, BAR_SFULL + 0));
-      if (n0 == 1) umma_commit_warp(bar_addr<D>(sbase, BAR_QEMPTY + 0));
+      if (n0 == j0 + 1) umma_commit_warp(bar_addr<D>(sbase, BAR_QEMPTY + 0));
     }
-    if (n1 > 0) {
+    if (n1 > j0) {
       issue_qk(1, k0);
       umma_commit_warp(bar_addr<D>(sbase, BAR_SFULL + 1));
-      if (n1 == 1) umma_commit_warp(bar_addr<D>(sbase, BAR_QEMPTY + 1));
+      if (n1 == j0 + 1) umma_commit_warp(bar_addr<D>(sbase, BAR_QEMPTY + 1));
     }
     umma_commit_warp(bar_addr<D>(sbase, BAR_KV + L::STAGES + k0));
 
-    for (int j = 0; j < nmax && ok; ++j) {
+    for (int j = j0; j < nmax && ok; ++j) {
       const int vs = st;
       const uint32_t vs_ph = kv_ph;
       if (++st == L::STAGES) { st = 0; kv_ph ^= 1; }
@@ -318,13 +320,13 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
         const int nt = t ? n1 : n0;
         if (j >= nt) continue;
         if (!(ok = wait_flip(BAR_PHALF + t, PH + t, 0))) break;
-        if (j > 0) {
+        if (j > j0) {
           if (!(ok = wait_flip(BAR_OCORR + t, OC + t, 0))) break;
         } else {
           if (!(ok = wait_flip(BAR_OFREE + t, OF + t, 1))) break;
         }
         tc_fence_after();
-        issue_pv_half(t, vs, 0, j > 0 ? 1u : 0u);
+        issue_pv_half(t, vs, 0, j > j0 ? 1u : 0u);
         if (!(ok = wait_flip(BAR_PFULL + t, PF + t, 0))) break;
         tc_fence_after();
         issue_pv_half(t, vs, 1, 1u);
@@ -492,14 +494,14 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
   int units_done = 0;
   Unit U;
   for (int it = 0; next_unit(p, it, U); ++it) {
-    if (U.n[t] == 0) continue;
+    if (!tile_active(U, t)) continue;
     const int row = U.mb[t] * BM + r;
     // l_e: sum of the unrounded P (gives LSE). l_o normalises O: l_e plus,
     // per K/V tile, the rounding error of that tile's largest P (the weight
     // that dominates a peaked row), so that O divides the P·V sum by a
     // denominator built from the same 16-bit weights where it matters.
     float m = -INFINITY, l_o = 0.f, l_e = 0.f;
-    for (int j = 0; j < U.n[t]; ++j) {
+    for (int j = U.j0; j < U.n[t]; ++j) {
       if (!wait_bar_warp(bar_addr<D>(sbase, BAR_SFULL + t), sf_ph, c)) return;
       sf_ph ^= 1;
       tc_fence_after();
@@ -523,7 +525,7 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
       // unchanged, P stays below 2^8 and the O rescale is skipped.
       const float m_new = (m_cand > m + RESCALE_THRESHOLD) ? m_cand : m;
       const float alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
-      if (j > 0) {
+      if (j > U.j0) {
         alpha_s[r] = alpha;
         mbar_arrive(bar_addr<D>(sbase, BAR_AFULL + t));
       }
@@ -579,7 +581,7 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
   Unit U;
   for (int it = 0; ok && next_unit(p, it, U); ++it) {
     // ---- rescale O_t for every K/V tile after the first
-    for (int j = 1; j < U.nmax && ok; ++j) {
+    for (int j = U.j0 + 1; j < U.nmax && ok; ++j) {
       for (int t = 0; t < 2; ++t) {
         if (j >= U.n[t]) continue;
         if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_AFULL + t), af_ph[t], c))) break;
@@ -611,7 +613,7 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
       const int row = U.mb[t] * BM + r;
       const int head = U.b * p.s.Hq + U.hq[t];
       float inv_l = 0.f, lse = -INFINITY;
-      const bool has = U.n[t] > 0;
+      const bool has = tile_active(U, t);
       if (has) {
         const int k = units_done[t]++, buf = k & 1;
         if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_STATS + 2 * t + buf), (k >> 1) & 1, c)))
@@ -627,6 +629,36 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
       }
       const int slab_row0 = U.mb[t] * BM + 32 * wl;
       const uint32_t t_o = tmem + (lane_base << 16) + TmemO<D>::col(t);
+      if (p.o_part != nullptr) {
+        // Split-KV: this split's O (normalised by its own l) and LSE, fp32,
+        // for the merge kernel; each thread writes its row's 128-byte chunks.
+        const size_t prow = ((size_t)U.split * p.s.B * p.s.Hq + head) * p.s.N + row;
+#pragma unroll 1
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t o[32];
+          if (has) {
+            tmem_ld_x32(t_o + 32 * q, o);
+            tmem_wait_ld();
+            reg_pin_x32(o);
+            if (q == D / 32 - 1) {
+              tc_fence_before();
+              mbar_arrive(bar_addr<D>(sbase, BAR_OFREE + t));
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = 0u;
+          }
+          if (row < p.s.N) {
+            float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D + 32 * q);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
+                                   __uint_as_float(o[4 * i + 2]) * inv_l, __uint_as_float(o[4 * i + 3]) * inv_l);
+          }
+        }
+        if (row < p.s.N) p.lse_part[prow] = lse;
+        continue;
+      }
 #pragma unroll 1
       for (int q = 0; q < D / 32; ++q) {
         uint32_t o[32];
@@ -764,6 +796,55 @@ __global__ void fa_wait_selftest_kernel(unsigned long long timeout_ns, int* out)
   }
 }
 
+// Split-KV merge: for each query row, combines the splits' partial results
+// (O_s normalised by its own denominator, LSE_s natural log; LSE_s = −inf for
+// a split with no allowed key) into O = Σ_s e^{LSE_s − m} O_s / Σ_s e^{LSE_s − m}
+// and LSE = m + ln Σ_s e^{LSE_s − m}, m = max_s LSE_s — one more step of the
+// online recurrence with a whole split as the tile. One warp per row, each
+// lane D/32 consecutive elements.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_merge_splits_kernel(const float* __restrict__ o_part,
+                                                              const float* __restrict__ lse_part,
+                                                              int splits, long long rows, void* o,
+                                                              float* lse) {
+  constexpr int E = D / 32;
+  const int lane = threadIdx.x & 31;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < rows;
+       row += nwarps) {
+    float m = -INFINITY;
+    for (int s = 0; s < splits; ++s) m = fmaxf(m, __ldg(lse_part + s * rows + row));
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    float l = 0.f;
+    if (m != -INFINITY) {
+      for (int s = 0; s < splits; ++s) {
+        const float ls = __ldg(lse_part + s * rows + row);
+        if (ls == -INFINITY) continue;
+        const float w = expf(ls - m);
+        l += w;
+        const float* src = o_part + ((long long)s * rows + row) * D + lane * E;
+        if constexpr (E == 4) {
+          const float4 x = __ldg(reinterpret_cast<const float4*>(src));
+          acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
+        } else {
+          const float2 x = __ldg(reinterpret_cast<const float2*>(src));
+          acc[0] += w * x.x; acc[1] += w * x.y;
+        }
+      }
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    uint32_t packed[E / 2];
+#pragma unroll
+    for (int e = 0; e < E / 2; ++e) packed[e] = cvt2<D, BF16>(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+    uint16_t* dst = reinterpret_cast<uint16_t*>(o) + row * D + lane * E;
+    if constexpr (E == 4) *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+    else *reinterpret_cast<uint32_t*>(dst) = packed[0];
+    if (lse != nullptr && lane == 0) lse[row] = l > 0.f ? m + logf(l) : -INFINITY;
+  }
+}
+
 // Evaluates the FMA-pipe exponential and ex2.approx on n inputs.
 __global__ void fa_exp2_selftest_kernel(const float* x, float* y_fma, float* y_mufu, int n) {
   const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
@@ -879,7 +960,7 @@ int make_map(CUtensorMap* map, const void* ptr, bool bf16, int d, int n, long lo
 
 template <int D, bool BF16>
 int launch(const void* q, const void* k, const void* v, void* o, const fa::Params& prm,
-           cudaStream_t stream, DeviceInfo& info, int slot) {
+           cudaStream_t stream, DeviceInfo& info, int slot, float* final_lse) {
   using L = fa::Layout<D>;
   auto kern = fa::fa_fwd_kernel<D, BF16>;
   {
@@ -914,7 +995,23 @@ int launch(const void* q, const void* k, const void* v, void* o, const fa::Param
   kern<<<grid, fa::NUM_THREADS, L::ALLOC, stream>>>(tq, tk, tv, to, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
+  if (prm.o_part != nullptr) {
+    const long long rows = (long long)s.B * s.Hq * s.N;
+    long long blocks = (rows + 7) / 8;
+    if (blocks > (long long)info.sms * 16) blocks = (long long)info.sms * 16;
+    fa::fa_merge_splits_kernel<D, BF16><<<(unsigned)blocks, 256, 0, stream>>>(
+        prm.o_part, prm.lse_part, s.splits, rows, o, final_lse);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "merge launch failed: %s", cudaGetErrorString(e));
+  }
   return FA_OK;
+}
+
+// Workspace of a split-KV call: partial O then partial LSE, fp32.
+size_t splitkv_bytes(long long heads_q, int N, int d, int splits) {
+  const size_t rows = (size_t)heads_q * N * (size_t)splits;
+  const size_t o_bytes = (rows * d * 4 + 255) / 256 * 256;
+  return o_bytes + (rows * 4 + 255) / 256 * 256;
 }
 
 }  // namespace
@@ -950,11 +1047,32 @@ int fa_unit_info(int B, int Hq, int Hk, int N, int causal, int u, int32_t* out) 
   return FA_OK;
 }
 
+int fa_unit_kv_range(int B, int Hq, int Hk, int N, int causal, int num_splits, int u,
+                     int key_len, int32_t* out) {
+  const int nu = fa_num_units(B, Hq, Hk, N, causal);
+  if (nu < 0) return nu;
+  if (num_splits < 1 || num_splits > 16) return fail(FA_ERR_INVALID_ARG, "num_splits out of [1, 16]");
+  if (out == nullptr || u < 0 || (long long)u >= (long long)nu * num_splits)
+    return fail(FA_ERR_INVALID_ARG, "bad unit index");
+  if (key_len < 0 || key_len > N) return fail(FA_ERR_INVALID_ARG, "key_len out of [0, N]");
+  const fa::Shape s = fa::make_shape(B, Hq, Hk, N, causal, num_splits);
+  fa::Unit U;
+  fa::decode_unit(s, u, U);
+  fa::resolve_unit(s, key_len, U);
+  const int32_t vals[12] = {U.b, U.hk, U.hq[0], U.mb[0], U.present[0], U.hq[1], U.mb[1],
+                            U.present[1], U.split, U.j0, U.n[0], U.n[1]};
+  memcpy(out, vals, sizeof(vals));
+  return FA_OK;
+}
+
 int fa_unit_for(int cta, int it, int grid) { return fa::unit_for(cta, it, grid); }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hk,
-           int N, int d, float scale, int causal, const int32_t* key_pad_lens, void* stream,
-           int dtype) {
+}  // extern "C"
+
+namespace {
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hk,
+             int N, int d, float scale, int causal, const int32_t* key_pad_lens, int splits,
+             void* workspace, size_t workspace_bytes, void* stream, int dtype) {
   g_err[0] = '\0';
   // ---- arguments that need no CUDA call
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr)
@@ -971,6 +1089,9 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   if (heads_q > 0x7fffffffLL || N > (1 << 30))
     return fail(FA_ERR_INVALID_ARG, "problem too large for 32-bit tile coordinates");
   if (fa_num_units(B, Hq, Hk, N, causal) < 0) return FA_ERR_INVALID_ARG;
+  if (splits < 1 || splits > 16) return fail(FA_ERR_INVALID_ARG, "num_splits %d out of [1, 16]", splits);
+  if ((long long)fa_num_units(B, Hq, Hk, N, causal) * splits > 0x7fffffffLL)
+    return fail(FA_ERR_INVALID_ARG, "too many work units");
   // ---- device and buffers
   if (!driver_fns().ok) return fail(FA_ERR_CUDA, "CUDA driver entry points unavailable");
   int dev = -1;
@@ -1011,17 +1132,64 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   fa::Params prm;
   prm.key_pad_lens = key_pad_lens;
   prm.lse = lse;
-  prm.s = fa::make_shape(B, Hq, Hk, N, causal);
+  prm.o_part = nullptr;
+  prm.lse_part = nullptr;
+  if (splits > 1) {
+    const size_t need = splitkv_bytes(heads_q, N, d, splits);
+    if (workspace_bytes < need)
+      return fail(FA_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", workspace_bytes, need);
+    if ((rc = check_range("workspace", workspace, need, 256)) != FA_OK) return rc;
+    const uintptr_t wb = reinterpret_cast<uintptr_t>(workspace), we = wb + need;
+    auto hits = [&](const void* x, size_t n) {
+      const uintptr_t xb = reinterpret_cast<uintptr_t>(x);
+      return x != nullptr && xb < we && wb < xb + n;
+    };
+    if (hits(q, q_bytes) || hits(k, kv_bytes) || hits(v, kv_bytes) || hits(o, q_bytes) ||
+        hits(lse, (size_t)heads_q * N * 4) || hits(key_pad_lens, (size_t)B * 4))
+      return fail(FA_ERR_INVALID_ARG, "workspace overlaps an argument");
+    const size_t rows = (size_t)heads_q * N * splits;
+    prm.o_part = reinterpret_cast<float*>(workspace);
+    prm.lse_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
+                                            (rows * d * 4 + 255) / 256 * 256);
+  }
+  prm.s = fa::make_shape(B, Hq, Hk, N, causal, splits);
   prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
   prm.timeout_ns = g_timeout_ns;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool bf16 = dtype == FA_BF16;
   if (d == 128)
-    return bf16 ? launch<128, true>(q, k, v, o, prm, st, info, 0)
-                : launch<128, false>(q, k, v, o, prm, st, info, 1);
-  return bf16 ? launch<64, true>(q, k, v, o, prm, st, info, 2)
-              : launch<64, false>(q, k, v, o, prm, st, info, 3);
+    return bf16 ? launch<128, true>(q, k, v, o, prm, st, info, 0, lse)
+                : launch<128, false>(q, k, v, o, prm, st, info, 1, lse);
+  return bf16 ? launch<64, true>(q, k, v, o, prm, st, info, 2, lse)
+              : launch<64, false>(q, k, v, o, prm, st, info, 3, lse);
 }
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hk,
+           int N, int d, float scale, int causal, const int32_t* key_pad_lens, void* stream,
+           int dtype) {
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hk, N, d, scale, causal, key_pad_lens, 1, nullptr, 0,
+                  stream, dtype);
+}
+
+size_t fa_splitkv_workspace_bytes(int B, int Hq, int N, int d, int num_splits) {
+  if (B < 1 || Hq < 1 || N < 1 || (d != 64 && d != 128) || num_splits < 1 || num_splits > 16)
+    return 0;
+  if (num_splits == 1) return 0;
+  return splitkv_bytes((long long)B * Hq, N, d, num_splits);
+}
+
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                   int Hk, int N, int d, float scale, int causal, const int32_t* key_pad_lens,
+                   int num_splits, void* workspace, size_t workspace_bytes, void* stream,
+                   int dtype) {
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hk, N, d, scale, causal, key_pad_lens, num_splits,
+                  workspace, workspace_bytes, stream, dtype);
+}
+
+
 
 int fa_get_device_status(void) {
   if (cudaDeviceSynchronize() != cudaSuccess)
