@@ -120,6 +120,47 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
  * arguments. */
 size_t fa_splitkv_workspace_bytes(int B, int Hq, int N, int d, int num_splits);
 
+/*
+ * fa_fwd_splitkv_static — fa_fwd_splitkv with the library's own scratch
+ * instead of a caller workspace, so the call allocates no memory at all.
+ * (The source pages have no counterpart: this is a calling convention of
+ * this library, not a step of the method.)
+ *
+ * Who needs it: callers that cannot allocate device memory per call and hold
+ * no pool to carve a workspace from, e.g. a server that reserved nearly all
+ * of HBM up front for weights and KV cache (an allocation there can fail in
+ * the middle of a request), or a latency-critical loop (cudaMalloc and
+ * cudaFree can synchronise the device and stall every stream), or a plain C
+ * caller that would otherwise have to keep a workspace alive across
+ * asynchronous calls.
+ *
+ * Scratch: one file-scope device array of FA_STATIC_SCRATCH_BYTES (32 MiB)
+ * per device, created when the library's module loads on that device. A
+ * problem whose split-KV workspace, fa_splitkv_workspace_bytes(B, Hq, N, d,
+ * num_splits), exceeds it is rejected with FA_ERR_INVALID_ARG and a message
+ * naming both sizes; nothing is launched. Nothing in the scratch has to start
+ * at zero: every partial result the merge reads is written earlier in the
+ * same call.
+ *
+ * Set-up: the first call on each device (with that device current) looks up
+ * the scratch's device address with cudaGetSymbolAddress, which may load the
+ * module on that device, and sets the kernel's attributes. Make that first
+ * call before any stream capture begins.
+ *
+ * Races: every call on a device shares that one scratch array. Two calls
+ * whose kernels can overlap (different streams, or host threads with no
+ * ordering between their streams) race on it and corrupt each other's
+ * results. Keep such calls on one stream, or use fa_fwd_splitkv with one
+ * workspace per stream.
+ *
+ * Arguments, results and errors as fa_fwd_splitkv, without the workspace.
+ */
+#define FA_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+int fa_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int Hq, int Hk, int N, int d, float scale, int causal,
+                          const int32_t* key_pad_lens, int num_splits, void* stream,
+                          int dtype);
+
 /* Message for the last error returned to the calling thread ("" if none).
  * The string is owned by the library (thread-local storage). */
 const char* fa_last_error_string(void);

@@ -47,6 +47,10 @@ def load_library(path=LIB_PATH):
                                  c_int, c_int, c_int, c_float, c_int, c_void_p, c_int, c_void_p,
                                  ctypes.c_size_t, c_void_p, c_int]
     L.fa_fwd_splitkv.restype = c_int
+    L.fa_fwd_splitkv_static.argtypes = [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                                        c_int, c_int, c_int, c_int, c_float, c_int, c_void_p,
+                                        c_int, c_void_p, c_int]
+    L.fa_fwd_splitkv_static.restype = c_int
     L.fa_splitkv_workspace_bytes.argtypes = [c_int] * 5
     L.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
     L.fa_unit_kv_range.argtypes = [c_int] * 8 + [ctypes.POINTER(ctypes.c_int32)]
@@ -160,6 +164,29 @@ def fa_fwd_splitkv(q, k, v, num_splits, causal=False, scale=None, key_pad_lens=N
                                  int(num_splits),
                                  workspace.data_ptr() if workspace is not None else None,
                                  ws_bytes, stream, _DTYPES[q.dtype]))
+    return (out, lse) if return_lse else out
+
+
+STATIC_SCRATCH_BYTES = 32 << 20  # FA_STATIC_SCRATCH_BYTES in include/fa.h
+
+
+def fa_fwd_splitkv_static(q, k, v, num_splits, causal=False, scale=None, key_pad_lens=None,
+                          out=None, lse=None, return_lse=True, stream=None):
+    """``fa_fwd_splitkv`` on the library's static scratch: the C call allocates
+    nothing (pass ``out`` and ``lse`` to allocate nothing here either).
+
+    Calls on one device share the scratch: calls whose kernels may overlap
+    (other streams) race on it. Problems whose split workspace exceeds
+    ``STATIC_SCRATCH_BYTES`` raise ``FaError``.
+    """
+    (B, Hq, Hk, N, d), out, lse, scale, stream = _prepare(q, k, v, key_pad_lens, out, lse,
+                                                          return_lse, scale, stream)
+    with torch.cuda.device(q.device):
+        check(lib.fa_fwd_splitkv_static(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                        lse.data_ptr() if lse is not None else None, B, Hq, Hk,
+                                        N, d, scale, 1 if causal else 0,
+                                        key_pad_lens.data_ptr() if key_pad_lens is not None
+                                        else None, int(num_splits), stream, _DTYPES[q.dtype]))
     return (out, lse) if return_lse else out
 
 
