@@ -20,6 +20,11 @@ What it computes, and where the pages say so (page title, then section):
   "坑四" (GQA/MQA: K and V carry fewer heads than Q).
 * [CSDN] aicoding.csdn.net page on ops-transformer FlashAttention, "第一层，
   算子融合": the mask is applied inside the fused kernel.
+* [CSDN] "第一层，算子融合" also lists Bias among the operations fused into
+  the kernel (beside Dropout and Mask), without giving its shape. Read here as
+  an additive term on the scaled scores, S = scale·Q Kᵀ + bias, with bias of
+  shape [Bb, Hb, N, N] broadcast over batch (Bb = 1) and heads (Hb = 1); the
+  mask applies after it.
 * [GQA] "深度探索Flash-Attention中GQA性能调优技术解析", section
   "num_splits参数的场景化配置": the attention work of one problem may be cut
   into num_splits parts. Read here as a split of the key range, each part's
@@ -66,14 +71,25 @@ def allowed_keys(rows, n_keys, causal, key_len):
     return ok
 
 
-def scores(q_rows, k, scale, ok):
-    """S = scale · Q Kᵀ for the given query rows, with −inf where not allowed.
+def scores(q_rows, k, scale, ok, bias_rows=None):
+    """S = scale · Q Kᵀ (+ bias) for the given query rows, −inf where not allowed.
 
-    [FA-VI]: the scores of standard attention; [CSDN]: the mask is part of the
-    same fused computation, taken here as an additive −inf.
+    [FA-VI]: the scores of standard attention; [CSDN]: the mask (and an
+    additive bias, not scaled) are part of the same fused computation, the
+    mask taken here as an additive −inf.
     """
     s = scale * (q_rows @ k.T)
+    if bias_rows is not None:
+        s = s + bias_rows
     return np.where(ok, s, -np.inf)
+
+
+def _bias_slice(bias, b, hq):
+    """The [N, N] bias plane of (b, hq): bias is [Bb, Hb, N, N] with Bb in {1, B}
+    and Hb in {1, Hq} (size-1 dimensions broadcast), or None."""
+    if bias is None:
+        return None
+    return bias[b if bias.shape[0] > 1 else 0, hq if bias.shape[1] > 1 else 0]
 
 
 def two_pass_softmax(s):
@@ -113,15 +129,17 @@ def _key_len(key_pad_lens, b, n):
     return int(min(max(int(key_pad_lens[b]), 0), n))
 
 
-def attention(q, k, v, scale, causal=False, key_pad_lens=None, row_block=1024):
+def attention(q, k, v, scale, causal=False, key_pad_lens=None, row_block=1024, bias=None):
     """Exact attention forward: returns (O [B,Hq,N,d], LSE [B,Hq,N]) in float64.
 
-    q: [B, Hq, N, d]; k, v: [B, Hk, N, d]; key_pad_lens: None or [B] integers.
+    q: [B, Hq, N, d]; k, v: [B, Hk, N, d]; key_pad_lens: None or [B] integers;
+    bias: None or [Bb, Hb, N, N] (see _bias_slice).
     Each row block holds full rows of S (all N keys), so the result is the
     plain definition of [FA-VI] with the two-pass softmax of [MCU] §二; the
     blocking over rows only bounds memory, as rows are independent.
     """
     q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    bias = None if bias is None else _as_f64(bias)
     B, Hq, N, d = q.shape
     Hk = k.shape[1]
     if Hq % Hk != 0:
@@ -133,16 +151,18 @@ def attention(q, k, v, scale, causal=False, key_pad_lens=None, row_block=1024):
         key_len = _key_len(key_pad_lens, b, N)
         for hq in range(Hq):
             hk = hq // group  # [NPU] "坑四": a K/V head serves Hq/Hk query heads
+            plane = _bias_slice(bias, b, hq)
             for r0 in range(0, N, row_block):
                 rows = np.arange(r0, min(r0 + row_block, N))
                 ok = allowed_keys(rows, N, causal, key_len)
-                s = scores(q[b, hq, rows], k[b, hk], scale, ok)
+                s = scores(q[b, hq, rows], k[b, hk], scale, ok,
+                           None if plane is None else plane[rows])
                 p, m, l = two_pass_softmax(s)
                 o[b, hq, rows], lse[b, hq, rows] = _finish(p, m, l, v[b, hk])
     return o, lse
 
 
-def attention_rows(q, k, v, scale, causal, key_pad_lens, picks):
+def attention_rows(q, k, v, scale, causal, key_pad_lens, picks, bias=None):
     """The same definition for selected rows only.
 
     picks: iterable of (b, hq, i). Returns (O [len(picks), d], LSE [len(picks)]).
@@ -157,7 +177,9 @@ def attention_rows(q, k, v, scale, causal, key_pad_lens, picks):
     for n, (b, hq, i) in enumerate(picks):
         hk = hq // group
         ok = allowed_keys([i], N, causal, _key_len(key_pad_lens, b, N))
-        s = scores(q[b, hq, [i]], k[b, hk], scale, ok)
+        plane = _bias_slice(bias, b, hq)
+        s = scores(q[b, hq, [i]], k[b, hk], scale, ok,
+                   None if plane is None else _as_f64(plane[[i]]))
         p, m, l = two_pass_softmax(s)
         o1, lse1 = _finish(p, m, l, v[b, hk])
         o[n], lse[n] = o1[0], lse1[0]

@@ -23,10 +23,11 @@ def rand(*shape, rng=RNG):
     return rng.standard_normal(shape)
 
 
-def brute_force(q, k, v, scale, causal, lens, key_lo=0, key_hi=None):
+def brute_force(q, k, v, scale, causal, lens, key_lo=0, key_hi=None, bias=None):
     """Scalar loops with math.fsum: one row at a time, no vectorised code.
 
-    Only keys key_lo <= j < key_hi take part (all keys by default)."""
+    Only keys key_lo <= j < key_hi take part (all keys by default); bias, if
+    given, is a full [B, Hq, N, N] array added to each score."""
     B, Hq, N, d = q.shape
     Hk = k.shape[1]
     G = Hq // Hk
@@ -42,7 +43,7 @@ def brute_force(q, k, v, scale, causal, lens, key_lo=0, key_hi=None):
                 if not keys:
                     continue
                 s = {j: scale * math.fsum(q[b, h, i, c] * k[b, kh, j, c] for c in range(d))
-                     for j in keys}
+                     + (0.0 if bias is None else bias[b, h, i, j]) for j in keys}
                 mx = max(s.values())
                 w = {j: math.exp(s[j] - mx) for j in keys}
                 tot = math.fsum(w.values())
@@ -398,6 +399,85 @@ def pin_merge_large_lse_stays_finite(orc):
     e = math.e
     close(o, [[e / (e + 1.0)]], 1e-14)
     close(lse, [800.0 + math.log1p(1.0 / e)], 1e-15)
+
+
+# ------------------------------------------------- additive bias ([CSDN] 第一层)
+
+def pin_bias_matches_scalar_brute_force(orc):
+    rng = np.random.default_rng(21)
+    q, k, v = rng.standard_normal((2, 2, 6, 3)), rng.standard_normal((2, 1, 6, 3)), \
+        rng.standard_normal((2, 1, 6, 2))
+    bias = 2.0 * rng.standard_normal((2, 2, 6, 6))
+    bias[0, 1, 2, 1] = -math.inf  # a bias of −inf removes that key
+    for causal, lens in itertools.product([False, True], [None, [4, 0]]):
+        o, lse = orc.attention(q, k, v, 0.8, causal, lens, bias=bias)
+        ob, lseb = brute_force(q, k, v, 0.8, causal, lens, bias=bias)
+        close(o, ob)
+        close(lse, lseb)
+
+
+def pin_bias_matches_torch_sdpa_float_mask(orc):
+    """torch's math SDPA adds a float attn_mask to the scaled scores."""
+    rng = np.random.default_rng(22)
+    B, Hq, Hk, N, d = 2, 4, 2, 19, 8
+    q, k, v = rng.standard_normal((B, Hq, N, d)), rng.standard_normal((B, Hk, N, d)), \
+        rng.standard_normal((B, Hk, N, d))
+    bias = rng.standard_normal((B, Hq, N, N))
+    o, _ = orc.attention(q, k, v, 0.4, True, None, bias=bias)
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    mask = torch.from_numpy(np.where(j <= i, bias, -np.inf))
+    kt = torch.from_numpy(k).repeat_interleave(Hq // Hk, dim=1)
+    vt = torch.from_numpy(v).repeat_interleave(Hq // Hk, dim=1)
+    with torch.nn.attention.sdpa_kernel(torch.nn.attention.SDPBackend.MATH):
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q), kt, vt, attn_mask=mask, scale=0.4).numpy()
+    close(o, ref, 1e-12)
+
+
+def pin_bias_constant_per_row_shifts_lse_only(orc):
+    rng = np.random.default_rng(23)
+    q, k, v = rng.standard_normal((1, 2, 9, 4)), rng.standard_normal((1, 2, 9, 4)), \
+        rng.standard_normal((1, 2, 9, 4))
+    c = rng.standard_normal((1, 2, 9, 1)) * 5.0
+    bias = np.broadcast_to(c, (1, 2, 9, 9)).copy()
+    o0, l0 = orc.attention(q, k, v, 0.5, True, [7])
+    o1, l1 = orc.attention(q, k, v, 0.5, True, [7], bias=bias)
+    close(o1, o0, 1e-12)
+    close(l1, l0 + c[..., 0], 1e-12)
+
+
+def pin_bias_minus_inf_equals_key_padding(orc):
+    rng = np.random.default_rng(24)
+    q, k, v = rng.standard_normal((2, 1, 8, 3)), rng.standard_normal((2, 1, 8, 3)), \
+        rng.standard_normal((2, 1, 8, 3))
+    lens = [5, 2]
+    bias = np.zeros((2, 1, 8, 8))
+    for b, L in enumerate(lens):
+        bias[b, :, :, L:] = -math.inf
+    o0, l0 = orc.attention(q, k, v, 0.9, False, lens)
+    o1, l1 = orc.attention(q, k, v, 0.9, False, None, bias=bias)
+    close(o1, o0, 1e-12)
+    close(l1, l0, 1e-12)
+
+
+def pin_bias_broadcast_equals_repeated(orc):
+    rng = np.random.default_rng(25)
+    B, Hq, N = 2, 3, 7
+    q, k, v = rng.standard_normal((B, Hq, N, 4)), rng.standard_normal((B, 1, N, 4)), \
+        rng.standard_normal((B, 1, N, 4))
+    for shape in [(1, 1), (1, Hq), (B, 1)]:
+        bias = rng.standard_normal(shape + (N, N))
+        full = np.broadcast_to(bias, (B, Hq, N, N)).copy()
+        o0, l0 = orc.attention(q, k, v, 0.7, True, None, bias=full)
+        o1, l1 = orc.attention(q, k, v, 0.7, True, None, bias=bias)
+        close(o1, o0, 1e-12)
+        close(l1, l0, 1e-12)
+        picks = [(b, h, i) for b in range(B) for h in range(Hq) for i in (0, 3, N - 1)]
+        orow, lrow = orc.attention_rows(q, k, v, 0.7, True, None, picks, bias=bias)
+        idx = tuple(np.array(picks).T)
+        close(orow, o0[idx], 1e-12)
+        close(lrow, l0[idx], 1e-12)
 
 
 def pin_hand_worked_golden(orc):

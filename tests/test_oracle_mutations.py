@@ -41,8 +41,8 @@ MUTATIONS = {
     "equations_l_local_factor_dropped": ("a_loc * p_loc.sum(axis=1)", "p_loc.sum(axis=1)"),
     "online_stale_max": ("m_new = np.maximum(m_old, s.max(axis=1))", "m_new = s.max(axis=1)"),
     "v_rows_reversed": ("rows] = _finish(p, m, l, v[b, hk])", "rows] = _finish(p, m, l, v[b, hk][::-1])"),
-    "k_rows_reversed": ("s = scores(q[b, hq, rows], k[b, hk], scale, ok)",
-                        "s = scores(q[b, hq, rows], k[b, hk][::-1], scale, ok)"),
+    "k_rows_reversed": ("s = scores(q[b, hq, rows], k[b, hk], scale, ok,",
+                        "s = scores(q[b, hq, rows], k[b, hk][::-1], scale, ok,"),
     "key_range_hi_inclusive": ("in_range = (j >= key_lo) & (j < key_hi)",
                                "in_range = (j >= key_lo) & (j <= key_hi)"),
     "key_range_lo_exclusive": ("in_range = (j >= key_lo) & (j < key_hi)",
@@ -52,6 +52,12 @@ MUTATIONS = {
     "merge_unweighted": ("num += w[..., None] * o_s", "num += o_s"),
     "merge_unnormalised": ("o[has] = num[has] / den[has][..., None]", "o[has] = num[has]"),
     "merge_lse_without_max": ("lse[has] = m[has] + np.log(den[has])", "lse[has] = np.log(den[has])"),
+    "bias_scaled": ("s = s + bias_rows", "s = s + scale * bias_rows"),
+    "bias_dropped": ("s = s + bias_rows", "s = s + 0.0 * bias_rows"),
+    "bias_transposed": ("None if plane is None else plane[rows])", "None if plane is None else plane.T[rows])"),
+    "bias_head_ignored": ("hq if bias.shape[1] > 1 else 0]", "0]"),
+    "bias_batch_ignored": ("b if bias.shape[0] > 1 else 0,", "0,"),
+    "bias_rows_wrong_row": ("_as_f64(plane[[i]])", "_as_f64(plane[[0]])"),
 }
 
 
