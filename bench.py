@@ -33,6 +33,7 @@ from tiled_online_softmax_03_b200.inputs import WORKLOADS, make_inputs  # noqa: 
 METRIC = ("attention fwd TFLOP/s (4·B·Hq·N²·d, ×½ causal) "
           "and % of B200 BF16 peak")
 FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0  # the same GEMM held under the 1 kW power cap
 KERNEL_SOURCES = ["tiled_online_softmax_03_b200/csrc/fa_fwd_sm100.cu",
                   "tiled_online_softmax_03_b200/csrc/fa_ptx.cuh",
                   "tiled_online_softmax_03_b200/csrc/fa_schedule.cuh"]
@@ -52,13 +53,16 @@ def kernel_hash():
 
 
 def peaks():
+    """(burst, sustained, source) dense bf16 TFLOP/s."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             m = json.load(f)
-        return float(m["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+        return float(m["bf16_tflops"]), float(m.get("bf16_tflops_sustained") or 0.0) or None, \
+            "measured (MEASURED_PEAKS.json)"
     except (OSError, KeyError, ValueError):
-        return FALLBACK_BF16_TFLOPS, "fallback (1.59 PFLOP/s, earlier measurement on this pool)"
+        return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS_SUSTAINED, \
+            "fallback (earlier measurement on this pool)"
 
 
 def recorded_traffic(workload):
@@ -91,14 +95,15 @@ class ClockSampler:
 
     def __init__(self, index):
         self.index = index
-        self.lines = []
+        self.lines = []  # (host time received, csv line)
         self.proc = None
+        self.window = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -109,7 +114,11 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, start, end):
+        """Host times bracketing the timed region (after synchronising)."""
+        self.window = (start, end)
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -121,26 +130,31 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
+        """Clocks, power and throttle reasons over the samples taken inside the
+        timed region (all samples if no region was marked)."""
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        for t, line in self.lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
                 s, m = float(parts[1]), float(parts[2])
+                pw = float(parts[3])
             except ValueError:
                 continue
-            sm.append(s)
-            mx = m
-            for n, flag in zip(names, parts[5:9]):
-                if flag.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+            rows.append((t, s, m, pw, [n for n, f in zip(names, parts[5:9]) if f.lower() == "active"]))
+        if self.window is not None:
+            inside = [r for r in rows if self.window[0] <= r[0] <= self.window[1]]
+            rows = inside or rows
+        if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        loaded = sorted(sm)[len(sm) // 4:] or sm  # drop the idle tail sampled at the edges
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        reasons = sorted({n for r in rows for n in r[4]})
+        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": rows[-1][2],
+                "sm_mhz_min": min(r[1] for r in rows),
+                "power_w_median": statistics.median(r[3] for r in rows),
+                "reasons": reasons, "samples": len(rows),
+                "window": "samples taken inside the timed region" if self.window else "all samples"}
 
 
 class OracleSampler:
@@ -283,6 +297,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--shape", default=None,
                     help="B,Hq,Hk,N[,causal] replacing the workload's shape (other settings kept)")
+    ap.add_argument("--bias", default="none", choices=["none", "heads", "full"],
+                    help="additive bias [1, Hq, N, N] (heads) or [B, Hq, N, N] (full), fa_fwd_bias")
     ap.add_argument("--splits", type=int, default=1,
                     help="K/V splits per Q tile pair (fa_fwd_splitkv; 1 = fa_fwd)")
     args = ap.parse_args()
@@ -334,8 +350,18 @@ def main():
         ws = torch.empty(binding.splitkv_workspace_bytes(w.B, w.Hq, w.N, w.d, args.splits),
                          dtype=torch.uint8, device=dev)
 
-    def call():
+    bias_t = None
+    if args.bias != "none":
         if args.splits > 1:
+            raise SystemExit("--bias and --splits > 1 cannot be combined")
+        from tiled_online_softmax_03_b200.inputs import make_bias
+        bias_t = make_bias(w, w.B if args.bias == "full" else 1, w.Hq, device=str(dev))
+
+    def call():
+        if bias_t is not None:
+            binding.fa_fwd_bias(q, k, v, bias_t, causal=w.causal, scale=w.scale, key_pad_lens=lens,
+                                out=o, lse=lse, stream=stream.cuda_stream)
+        elif args.splits > 1:
             binding.fa_fwd_splitkv(q, k, v, args.splits, causal=w.causal, scale=w.scale,
                                    key_pad_lens=lens, out=o, lse=lse, workspace=ws,
                                    stream=stream.cuda_stream)
@@ -361,6 +387,7 @@ def main():
     with ClockSampler(local) as clocks:
         barrier()
         torch.cuda.synchronize()
+        host_t0 = time.time()
         t_begin.record(stream)
         for i in range(args.steps):
             if flush is not None:
@@ -370,17 +397,21 @@ def main():
             ends[i].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
+        clocks.mark(host_t0, time.time())
         barrier()
     status = binding.device_status()
-    total_ms = rank_max(t_begin.elapsed_time(t_end))
     kern_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     kern_avg = rank_max(sum(kern_ms) / len(kern_ms))
+    # With an L2 flush between steps the loop also times the flush writes,
+    # which are not part of the job: the steps' own event times count instead.
+    total_ms = rank_max(t_begin.elapsed_time(t_end)) if flush is None else kern_avg * args.steps
 
     # ---- end-to-end through the public API: pinned host inputs in, O and LSE out
     hq_, hk_, hv_ = (x[n].pin_memory() for n in ("q", "k", "v"))
     ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
     hlens = x["key_pad_lens"].pin_memory() if x["key_pad_lens"] is not None else None
+    hbias = bias_t.cpu().pin_memory() if bias_t is not None else None
     e2e_steps = max(1, min(args.e2e_steps, args.steps))
 
     def e2e_step():
@@ -389,6 +420,8 @@ def main():
         v.copy_(hv_, non_blocking=True)
         if hlens is not None:
             lens.copy_(hlens, non_blocking=True)
+        if hbias is not None:
+            bias_t.copy_(hbias, non_blocking=True)
         call()
         ho.copy_(o, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
@@ -405,7 +438,8 @@ def main():
     barrier()
     e2e_ms = rank_max(e0.elapsed_time(e1)) / e2e_steps
     h2d = sum(t.numel() * t.element_size() for t in (hq_, hk_, hv_)) + \
-        (hlens.numel() * 4 if hlens is not None else 0)
+        (hlens.numel() * 4 if hlens is not None else 0) + \
+        (hbias.numel() * hbias.element_size() if hbias is not None else 0)
     d2h = ho.numel() * ho.element_size() + hl.numel() * 4
 
     if world > 1:
@@ -416,14 +450,24 @@ def main():
     f = flops(w)
     ms_per_step = total_ms / args.steps
     value = whole_job_tflops(f, world, ms_per_step)
-    peak, peak_src = peaks()
+    clk = clocks.summary()
+    burst, sustained, peak_src = peaks()
+    # Burst peak for a kernel timed before the power cap engages; the sustained
+    # one once the timed region ran under sw_power_cap (a long back-to-back loop).
+    capped = "sw_power_cap" in clk.get("reasons", [])
+    peak = sustained if (capped and sustained) else burst
+    peak_src += ", sustained (sw_power_cap active in the timed region)" if peak == sustained and capped \
+        else ", burst"
     achieved = f / (kern_avg * 1e-3) / 1e12
-    traffic = recorded_traffic(w.name) if args.splits == 1 else None
+    traffic = recorded_traffic(w.name) if args.splits == 1 and args.bias == "none" else None
     config = config_of(w, world)
     kernels = "fa_fwd_kernel"
     if args.splits > 1:
         config["num_splits"] = args.splits
         kernels = "fa_fwd_kernel + fa_merge_splits_kernel"
+    if bias_t is not None:
+        config["bias"] = list(bias_t.shape)
+        kernels = "fa_fwd_kernel (bias)"
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -432,13 +476,14 @@ def main():
         "config": config,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                     "frac_of_burst": achieved / burst,
                      "kernel": kernels, "kernel_ms": kern_avg,
                      "flop_per_launch": f},
         "e2e": {"value": whole_job_tflops(f, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "steps": e2e_steps},
         "gpu_launches": args.steps * (2 if args.splits > 1 else 1),
-        "clocks": clocks.summary(),
+        "clocks": clk,
         "device_status": status,
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -115,6 +115,31 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
                    const int32_t* key_pad_lens, int num_splits, void* workspace,
                    size_t workspace_bytes, void* stream, int dtype);
 
+/*
+ * fa_fwd_bias — fa_fwd with an additive bias on the scaled scores:
+ *     S = scale · Q Kᵀ + bias + mask,  O = softmax_rows(S) · V,  LSE = ln Σ_j e^{S_ij}.
+ * (The CSDN ops-transformer page, section "第一层，算子融合", lists Bias among
+ * the operations fused into the attention kernel; its shape is not given
+ * there. The bias is not multiplied by scale; the mask applies after it.)
+ *
+ *   bias          device pointer, 16-byte aligned, dtype `dtype`, contiguous
+ *                 [bias_B, bias_H, N, N]: row i, column j is added to the score
+ *                 of query i and key j. Finite values or −inf (which removes
+ *                 that key for that query); +inf or NaN give undefined results.
+ *   bias_B        1 (shared by every batch) or B.
+ *   bias_H        1 (shared by every query head) or Hq.
+ *   other arguments as for fa_fwd.
+ * N must be a multiple of 8 (each bias row is loaded by TMA, which needs
+ * 16-byte row strides); other N return FA_ERR_UNSUPPORTED. The bias must not
+ * overlap o or lse. Each launch reads the bias blocks of the visited tiles
+ * from HBM once per Q tile: B·Hq·N² elements for a full bias (about half
+ * with causal), fewer when it is broadcast and L2 catches the reuse.
+ * Returns FA_OK or a negative fa_status, as fa_fwd.
+ */
+int fa_fwd_bias(const void* q, const void* k, const void* v, const void* bias, int bias_B,
+                int bias_H, void* o, float* lse, int B, int Hq, int Hk, int N, int d, float scale,
+                int causal, const int32_t* key_pad_lens, void* stream, int dtype);
+
 /* Workspace bytes fa_fwd_splitkv needs: B·Hq·N·num_splits·(d + 1) floats,
  * each part rounded up to 256 bytes; 0 for num_splits == 1 and for invalid
  * arguments. */

@@ -176,3 +176,14 @@ def test_split_count_and_workspace_size():
         binding.unit_kv_range(1, 1, 1, 128, 0, 2, 2, 128)  # only units 0 and 1 exist
     with pytest.raises(binding.FaError):
         binding.unit_kv_range(1, 1, 1, 128, 0, 2, 0, 129)  # key_len > N
+
+
+def test_bias_arguments_rejected_before_cuda():
+    lib = binding.lib
+    # bias_B must be 1 or B, bias_H 1 or Hq; N % 8 != 0 is unsupported; NULL bias rejected
+    args = lambda bias, bB, bH, N: (16, 16, 16, bias, bB, bH, 16, None, 2, 4, 2, N, 64, 0.1, 0,  # noqa: E731
+                                    None, None, 1)
+    assert lib.fa_fwd_bias(*args(16, 3, 1, 64)) == -1 and "batch" in binding.last_error()
+    assert lib.fa_fwd_bias(*args(16, 1, 2, 64)) == -1 and "head" in binding.last_error()
+    assert lib.fa_fwd_bias(*args(16, 2, 4, 60)) == -2 and "N % 8" in binding.last_error()
+    assert lib.fa_fwd_bias(*args(None, 1, 1, 64)) == -1 and "NULL" in binding.last_error()

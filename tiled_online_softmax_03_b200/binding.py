@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["FaError", "fa_fwd", "fa_fwd_splitkv", "splitkv_workspace_bytes", "load_library", "lib", "FA_OK", "FA_ERR_INVALID_ARG",
+__all__ = ["FaError", "fa_fwd", "fa_fwd_bias", "fa_fwd_splitkv", "splitkv_workspace_bytes", "load_library", "lib", "FA_OK", "FA_ERR_INVALID_ARG",
            "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT"]
 
 FA_OK = 0
@@ -43,6 +43,10 @@ def load_library(path=LIB_PATH):
     L.fa_fwd.argtypes = [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                          c_int, c_int, c_float, c_int, c_void_p, c_void_p, c_int]
     L.fa_fwd.restype = c_int
+    L.fa_fwd_bias.argtypes = [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p,
+                              c_void_p, c_int, c_int, c_int, c_int, c_int, c_float, c_int,
+                              c_void_p, c_void_p, c_int]
+    L.fa_fwd_bias.restype = c_int
     L.fa_fwd_splitkv.argtypes = [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int,
                                  c_int, c_int, c_int, c_float, c_int, c_void_p, c_int, c_void_p,
                                  ctypes.c_size_t, c_void_p, c_int]
@@ -131,6 +135,29 @@ def fa_fwd(q, k, v, causal=False, scale=None, key_pad_lens=None, out=None, lse=N
                          scale, 1 if causal else 0,
                          key_pad_lens.data_ptr() if key_pad_lens is not None else None,
                          stream, _DTYPES[q.dtype]))
+    return (out, lse) if return_lse else out
+
+
+def fa_fwd_bias(q, k, v, bias, causal=False, scale=None, key_pad_lens=None, out=None, lse=None,
+                return_lse=True, stream=None):
+    """``fa_fwd`` with an additive bias on the scaled scores.
+
+    ``bias`` is a contiguous CUDA tensor [Bb, Hb, N, N] of q's dtype with Bb in
+    {1, B} and Hb in {1, Hq}; it is added to scale·QKᵀ before the mask.
+    """
+    (B, Hq, Hk, N, d), out, lse, scale, stream = _prepare(q, k, v, key_pad_lens, out, lse,
+                                                          return_lse, scale, stream)
+    if not bias.is_cuda or not bias.is_contiguous() or bias.dim() != 4 or \
+            bias.dtype != q.dtype or tuple(bias.shape[2:]) != (N, N):
+        raise FaError(FA_ERR_INVALID_ARG,
+                      "bias must be a contiguous [Bb, Hb, N, N] CUDA tensor of q's dtype")
+    with torch.cuda.device(q.device):
+        check(lib.fa_fwd_bias(q.data_ptr(), k.data_ptr(), v.data_ptr(), bias.data_ptr(),
+                              bias.shape[0], bias.shape[1], out.data_ptr(),
+                              lse.data_ptr() if lse is not None else None, B, Hq, Hk, N, d,
+                              scale, 1 if causal else 0,
+                              key_pad_lens.data_ptr() if key_pad_lens is not None else None,
+                              stream, _DTYPES[q.dtype]))
     return (out, lse) if return_lse else out
 
 

@@ -17,7 +17,8 @@
 //   warps 8-11  correction (rescale O in TMEM) and epilogue (O/l, LSE, stores)
 //   warp 12     tcgen05.mma issue (one thread)
 //   warp 13     TMA loads (one thread)
-//   warps 14-15 no work
+//   warps 14-15 bias mode: TMA loads of the bias tiles of Q tile 0 / 1
+//                (one thread each); otherwise no work
 // Per K/V tile j and Q tile t the MMA thread issues S_t = Q_t·K_jᵀ into TMEM,
 // the softmax warps turn S_t into P_t (16-bit, written over S_t in TMEM) and
 // the running statistics, the correction warps rescale O_t, and the MMA thread
@@ -72,25 +73,34 @@ enum {
   BAR_STATS = 16,   // [2 tiles][2 buffers] softmax -> epilogue: final m, l in smem
   BAR_DRAIN = 20,   // MMA drain on the abort path
   BAR_PHALF = 21,   // [2] softmax -> MMA: P of the first 64 keys written to TMEM
-  BAR_KV = 23       // [STAGES] full, then [STAGES] empty
+  BAR_BFULL = 23,   // [2] TMA -> softmax: bias tile loaded (bias mode)
+  BAR_BEMPTY = 25,  // [2] softmax -> TMA: bias tile read
+  BAR_KV = 27       // [STAGES] full, then [STAGES] empty
 };
 
-template <int D>
+// Shared memory: barriers and flags first, then 1 KB-aligned tiles. With an
+// additive bias the K/V ring is halved to make room for one 128×128 16-bit
+// bias tile per Q tile.
+template <int D, bool BIAS = false>
 struct Layout {
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int STAGES = (D == 128) ? 4 : 8;
-  static constexpr int OFF_Q = 0;
+  static constexpr int STAGES = BIAS ? ((D == 128) ? 2 : 4) : ((D == 128) ? 4 : 8);
+  static constexpr int BIAS_BYTES = BIAS ? BM * BN * 2 : 0;
+  static constexpr int NUM_BARS = BAR_KV + 2 * STAGES;
+  static constexpr int OFF_BAR = 0;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;     // tmem base, abort flag
+  static constexpr int OFF_Q = 1024;
   static constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;
-  static constexpr int OFF_OST = OFF_KV + STAGES * KV_BYTES;
+  static constexpr int OFF_BIAS = OFF_KV + STAGES * KV_BYTES;  // [2 tiles] bias mode only
+  static constexpr int OFF_OST = OFF_BIAS + 2 * BIAS_BYTES;
   static constexpr int OFF_ALPHA = OFF_OST + 8 * OST_BYTES;   // [2 tiles][128] float
   static constexpr int OFF_STATS = OFF_ALPHA + 2 * BM * 4;    // [2 buf][2 tiles][128] float4
-  static constexpr int OFF_BAR = OFF_STATS + 2 * 2 * BM * 16;
-  static constexpr int NUM_BARS = BAR_KV + 2 * STAGES;
-  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;     // tmem base, abort flag
-  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int BYTES = OFF_STATS + 2 * 2 * BM * 16;
   static constexpr int ALLOC = BYTES + 1024;                  // base is rounded up to 1 KB
-  static_assert(OFF_KV % 1024 == 0 && OFF_OST % 2048 == 0, "tile alignment");
+  static_assert(OFF_MISC + 16 <= OFF_Q, "barrier area");
+  static_assert(OFF_KV % 1024 == 0 && OFF_BIAS % 1024 == 0 && OFF_OST % 1024 == 0,
+                "tile alignment");
   static_assert(ALLOC <= 232448, "shared memory budget");
 };
 
@@ -99,6 +109,9 @@ struct Params {
   float* lse;
   float* o_part;    // split-KV: [splits][B·Hq][N][d] fp32 partial O (normalised), else null
   float* lse_part;  // split-KV: [splits][B·Hq][N] fp32 partial LSE
+  int bias_bmul;    // bias mode: bias plane of (b, hq) is (b·bias_bmul)·bias_H + hq·bias_hmul
+  int bias_hmul;
+  int bias_H;
   Shape s;
   float scale_log2;
   unsigned long long timeout_ns;
@@ -148,9 +161,8 @@ __device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, con
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int D>
 __device__ __forceinline__ uint32_t bar_addr(uint32_t sbase, int i) {
-  return sbase + Layout<D>::OFF_BAR + 8 * i;
+  return sbase + 8 * i;  // barriers sit at the start of shared memory in every layout
 }
 
 __device__ __forceinline__ int key_len_of(const Params& p, int b) {
@@ -168,10 +180,10 @@ __device__ __forceinline__ bool next_unit(const Params& p, int it, Unit& U) {
 }
 
 // ============================================================ TMA producer
-template <int D>
+template <int D, bool BIAS>
 __device__ void role_load(const Params& p, uint32_t sbase, const Ctl& c, const CUtensorMap* tm_q,
                           const CUtensorMap* tm_k, const CUtensorMap* tm_v) {
-  using L = Layout<D>;
+  using L = Layout<D, BIAS>;
   uint32_t qe_ph[2] = {0, 0};
   int st = 0;
   uint32_t kv_ph = 0;
@@ -182,9 +194,9 @@ __device__ void role_load(const Params& p, uint32_t sbase, const Ctl& c, const C
   for (int it = 0; ok && next_unit(p, it, U); ++it) {
     for (int t = 0; t < 2 && ok; ++t) {
       if (!tile_active(U, t)) continue;
-      if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_QEMPTY + t), qe_ph[t] ^ 1, c))) break;
+      if (!(ok = wait_bar(bar_addr(sbase, BAR_QEMPTY + t), qe_ph[t] ^ 1, c))) break;
       qe_ph[t] ^= 1;
-      const uint32_t full = bar_addr<D>(sbase, BAR_QFULL + t);
+      const uint32_t full = bar_addr(sbase, BAR_QFULL + t);
       mbar_arrive_expect_tx(full, L::Q_BYTES);
       last_q_ph[t] = (armed_q >> t & 1) ? last_q_ph[t] ^ 1 : 0;
       armed_q |= 1u << t;
@@ -196,8 +208,8 @@ __device__ void role_load(const Params& p, uint32_t sbase, const Ctl& c, const C
     const int kv_head = U.b * p.s.Hk + U.hk;
     for (int j = U.j0; j < U.nmax && ok; ++j) {
       for (int which = 0; which < 2; ++which) {  // K_j then V_j
-        if (!(ok = wait_bar(bar_addr<D>(sbase, BAR_KV + L::STAGES + st), kv_ph ^ 1, c))) break;
-        const uint32_t full = bar_addr<D>(sbase, BAR_KV + st);
+        if (!(ok = wait_bar(bar_addr(sbase, BAR_KV + L::STAGES + st), kv_ph ^ 1, c))) break;
+        const uint32_t full = bar_addr(sbase, BAR_KV + st);
         mbar_arrive_expect_tx(full, L::KV_BYTES);
         last_kv_ph[st] = kv_ph;
         armed_kv |= 1u << st;
@@ -218,18 +230,53 @@ __device__ void role_load(const Params& p, uint32_t sbase, const Ctl& c, const C
     volatile int no_abort = 0;
     drain.abort_flag = &no_abort;
     for (int t = 0; t < 2; ++t)
-      if (armed_q >> t & 1) wait_bar(bar_addr<D>(sbase, BAR_QFULL + t), last_q_ph[t], drain);
+      if (armed_q >> t & 1) wait_bar(bar_addr(sbase, BAR_QFULL + t), last_q_ph[t], drain);
     for (int s = 0; s < L::STAGES; ++s)
-      if (armed_kv >> s & 1) wait_bar(bar_addr<D>(sbase, BAR_KV + s), last_kv_ph[s], drain);
+      if (armed_kv >> s & 1) wait_bar(bar_addr(sbase, BAR_KV + s), last_kv_ph[s], drain);
   }
 }
 
 // ============================================================= MMA issuer
+// Bias tiles for Q tile t (bias mode; one thread each of warps 14 and 15):
+// for every K/V tile j the tile visits, the 128×128 block of the bias plane
+// at rows of the Q tile and keys of K/V tile j, as two 64-column boxes with
+// the 128-byte swizzle, into the tile's single bias buffer. Rows and keys
+// past N read as zero (they are masked or never stored).
+template <int D>
+__device__ void role_bias_load(const Params& p, uint32_t sbase, const Ctl& c,
+                               const CUtensorMap* tm_b, int t) {
+  using L = Layout<D, true>;
+  uint32_t be_ph = 0, last_ph = 0;
+  bool armed = false, ok = true;
+  Unit U;
+  for (int it = 0; ok && next_unit(p, it, U); ++it) {
+    if (!tile_active(U, t)) continue;
+    const int plane = U.b * p.bias_bmul * p.bias_H + U.hq[t] * p.bias_hmul;
+    for (int j = U.j0; j < U.n[t] && ok; ++j) {
+      if (!(ok = wait_bar(bar_addr(sbase, BAR_BEMPTY + t), be_ph ^ 1, c))) break;
+      be_ph ^= 1;
+      const uint32_t full = bar_addr(sbase, BAR_BFULL + t);
+      mbar_arrive_expect_tx(full, L::BIAS_BYTES);
+      last_ph = armed ? last_ph ^ 1 : 0;
+      armed = true;
+      for (int bx = 0; bx < BN / 64; ++bx)
+        tma_load_3d(sbase + L::OFF_BIAS + t * L::BIAS_BYTES + bx * SW128_BOX_BYTES, tm_b,
+                    j * BN + bx * 64, U.mb[t] * BM, plane, full);
+    }
+  }
+  if (!ok && armed) {
+    // Let the armed copy land before the CTA can exit (bounded, short).
+    volatile int no_abort = 0;
+    Ctl drain{&no_abort, 100000000ull};
+    wait_bar(bar_addr(sbase, BAR_BFULL + t), last_ph, drain);
+  }
+}
+
 // Run by the whole of warp 12, converged; one elected lane issues each
 // tcgen05 instruction.
-template <int D, bool BF16>
+template <int D, bool BF16, bool BIAS>
 __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const Ctl& c) {
-  using L = Layout<D>;
+  using L = Layout<D, BIAS>;
   constexpr uint32_t IDESC_QK = idesc_f16(BF16, BN, false);  // S = Q·Kᵀ, both K-major
   constexpr uint32_t IDESC_PV = idesc_f16(BF16, D, true);    // O += P·V, V is MN-major
   int st = 0;
@@ -274,7 +321,7 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
   constexpr uint32_t QF = 0, PF = 2, OC = 4, OF = 6, PH = 8;
   uint32_t ph = 0;
   auto wait_flip = [&](int bar, uint32_t bit, uint32_t invert) {
-    const bool r = wait_bar_warp(bar_addr<D>(sbase, bar), ((ph >> bit) & 1u) ^ invert, c);
+    const bool r = wait_bar_warp(bar_addr(sbase, bar), ((ph >> bit) & 1u) ^ invert, c);
     ph ^= 1u << bit;
     return r;
   };
@@ -285,7 +332,7 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
     const int k0 = st;
     const uint32_t k0_ph = kv_ph;
     if (++st == L::STAGES) { st = 0; kv_ph ^= 1; }
-    if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_KV + k0), k0_ph, c))) break;
+    if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_KV + k0), k0_ph, c))) break;
     if (n0 > j0 && !(ok = wait_flip(BAR_QFULL + 0, QF + 0, 0))) break;
     if (n1 > j0 && !(ok = wait_flip(BAR_QFULL + 1, QF + 1, 0))) break;
     tc_fence_after();
@@ -293,15 +340,15 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
     // so the next unit's Q tile loads while this unit's softmax and P·V run.
     if (n0 > j0) {
       issue_qk(0, k0);
-      umma_commit_warp(bar_addr<D>(sbase, BAR_SFULL + 0));
-      if (n0 == j0 + 1) umma_commit_warp(bar_addr<D>(sbase, BAR_QEMPTY + 0));
+      umma_commit_warp(bar_addr(sbase, BAR_SFULL + 0));
+      if (n0 == j0 + 1) umma_commit_warp(bar_addr(sbase, BAR_QEMPTY + 0));
     }
     if (n1 > j0) {
       issue_qk(1, k0);
-      umma_commit_warp(bar_addr<D>(sbase, BAR_SFULL + 1));
-      if (n1 == j0 + 1) umma_commit_warp(bar_addr<D>(sbase, BAR_QEMPTY + 1));
+      umma_commit_warp(bar_addr(sbase, BAR_SFULL + 1));
+      if (n1 == j0 + 1) umma_commit_warp(bar_addr(sbase, BAR_QEMPTY + 1));
     }
-    umma_commit_warp(bar_addr<D>(sbase, BAR_KV + L::STAGES + k0));
+    umma_commit_warp(bar_addr(sbase, BAR_KV + L::STAGES + k0));
 
     for (int j = j0; j < nmax && ok; ++j) {
       const int vs = st;
@@ -314,7 +361,7 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
         kn_ph = kv_ph;
         if (++st == L::STAGES) { st = 0; kv_ph ^= 1; }
       }
-      if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_KV + vs), vs_ph, c))) break;
+      if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_KV + vs), vs_ph, c))) break;
       bool kn_ready = false;
       for (int t = 0; t < 2; ++t) {
         const int nt = t ? n1 : n0;
@@ -331,29 +378,29 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
         tc_fence_after();
         issue_pv_half(t, vs, 1, 1u);
         if (j == nt - 1) {
-          umma_commit_warp(bar_addr<D>(sbase, BAR_PVDONE + t));
+          umma_commit_warp(bar_addr(sbase, BAR_PVDONE + t));
         } else {
           if (!kn_ready) {
-            if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_KV + kn), kn_ph, c))) break;
+            if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_KV + kn), kn_ph, c))) break;
             kn_ready = true;
             tc_fence_after();
           }
           issue_qk(t, kn);
-          umma_commit_warp(bar_addr<D>(sbase, BAR_SFULL + t));
-          if (j + 2 == nt) umma_commit_warp(bar_addr<D>(sbase, BAR_QEMPTY + t));
+          umma_commit_warp(bar_addr(sbase, BAR_SFULL + t));
+          if (j + 2 == nt) umma_commit_warp(bar_addr(sbase, BAR_QEMPTY + t));
         }
       }
       if (!ok) break;
-      umma_commit_warp(bar_addr<D>(sbase, BAR_KV + L::STAGES + vs));
-      if (kn >= 0) umma_commit_warp(bar_addr<D>(sbase, BAR_KV + L::STAGES + kn));
+      umma_commit_warp(bar_addr(sbase, BAR_KV + L::STAGES + vs));
+      if (kn >= 0) umma_commit_warp(bar_addr(sbase, BAR_KV + L::STAGES + kn));
     }
   }
   if (!ok) {
     // Let every issued MMA finish before TMEM is released.
     volatile int no_abort = 0;
     Ctl drain{&no_abort, 100000000ull};
-    umma_commit_warp(bar_addr<D>(sbase, BAR_DRAIN));
-    wait_bar_warp(bar_addr<D>(sbase, BAR_DRAIN), 0, drain);
+    umma_commit_warp(bar_addr(sbase, BAR_DRAIN));
+    wait_bar_warp(bar_addr(sbase, BAR_DRAIN), 0, drain);
   }
 }
 
@@ -402,23 +449,18 @@ constexpr int EXP2_FMA_EVERY = 1 << 30;  // off: slower than ex2.approx alone in
 // Row max of one S tile for this thread's row, in log2 units of the scaled
 // score. MASKED: keys c >= nvalid are masked, and s is rewritten in place to
 // s·scale·log2e (−inf where masked); otherwise s stays raw and the max of the
-// scaled row is taken as max(s)·k for k >= 0, min(s)·k for k < 0.
+// scaled row is max(s)·k, valid for k >= 0 (a negative scale always takes
+// the masked form, with every key of an interior tile valid).
 template <bool MASKED>
 __device__ __forceinline__ float row_max(uint32_t (&s)[BN], float sl2, int nvalid) {
   float mx[8];
   if constexpr (!MASKED) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(s[i]);
-    if (sl2 >= 0.f) {
-#pragma unroll
-      for (int i = 8; i < BN; i += 2)
-        mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
-      return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl2;
-    }
 #pragma unroll
     for (int i = 8; i < BN; i += 2)
-      mx[(i >> 1) & 7] = fmin3(mx[(i >> 1) & 7], __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
-    return fmin3(fmin3(mx[0], mx[1], mx[2]), fmin3(mx[3], mx[4], mx[5]), fminf(mx[6], mx[7])) * sl2;
+      mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
+    return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl2;
   } else {
 #pragma unroll
     for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
@@ -432,6 +474,43 @@ __device__ __forceinline__ float row_max(uint32_t (&s)[BN], float sl2, int nvali
     }
     return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
   }
+}
+
+// Bias mode: s·scale·log2e + bias·log2e for this thread's row, −inf for keys
+// c >= nvalid, written over s; returns the row max (log2 units). brow is the
+// row in the bias buffer (first 64-column box); its 16-byte chunks sit at
+// chunk ^ (row & 7), the 128-byte swizzle the TMA load applied.
+template <bool BF16>
+__device__ __forceinline__ float row_max_bias(uint32_t (&s)[BN], float sl2, int nvalid,
+                                              const uint8_t* brow, int sw) {
+  constexpr float LOG2E = 1.4426950408889634f;
+  float mx[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < BN / 8; ++c) {
+    const uint4 bv = *reinterpret_cast<const uint4*>(brow + (c >> 3) * SW128_BOX_BYTES +
+                                                     (((c & 7) ^ sw) << 4));
+    const uint32_t w[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = c * 8 + 2 * e;
+      float b0, b1;
+      if constexpr (BF16) {
+        b0 = __uint_as_float(w[e] << 16);
+        b1 = __uint_as_float(w[e] & 0xffff0000u);
+      } else {
+        b0 = __half2float(__ushort_as_half((unsigned short)(w[e] & 0xffffu)));
+        b1 = __half2float(__ushort_as_half((unsigned short)(w[e] >> 16)));
+      }
+      const float v0 = i < nvalid ? fmaf(__uint_as_float(s[i]), sl2, b0 * LOG2E) : -INFINITY;
+      const float v1 = i + 1 < nvalid ? fmaf(__uint_as_float(s[i + 1]), sl2, b1 * LOG2E) : -INFINITY;
+      s[i] = __float_as_uint(v0);
+      s[i + 1] = __float_as_uint(v1);
+      mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], v0, v1);
+    }
+  }
+  return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
 }
 
 // P = exp2(s·scale·log2e − mref) for this thread's row, rounded to 16 bits and
@@ -480,18 +559,19 @@ __device__ __forceinline__ float round16(float x) {
   else return __half2float(__float2half_rn(x));
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool BIAS>
 __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uint32_t tmem,
                              const Ctl& c, int t) {
-  using L = Layout<D>;
+  using L = Layout<D, BIAS>;
   const int r = threadIdx.x & 127;                           // row within the Q tile
   const uint32_t lane_base = (uint32_t)((threadIdx.x >> 5) & 3) * 32;
   const uint32_t t_s = tmem + (lane_base << 16) + S_COL[t];  // this warp's lanes of S_t / P_t
   float* alpha_s = reinterpret_cast<float*>(smem + L::OFF_ALPHA) + t * BM;
   float4* stats = reinterpret_cast<float4*>(smem + L::OFF_STATS);
   const float sl2 = p.scale_log2;
-  uint32_t sf_ph = 0;
+  uint32_t sf_ph = 0, bf_ph = 0;
   int units_done = 0;
+  const uint8_t* brow = smem + L::OFF_BIAS + t * L::BIAS_BYTES + r * 128;
   Unit U;
   for (int it = 0; next_unit(p, it, U); ++it) {
     if (!tile_active(U, t)) continue;
@@ -502,7 +582,7 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
     // denominator built from the same 16-bit weights where it matters.
     float m = -INFINITY, l_o = 0.f, l_e = 0.f;
     for (int j = U.j0; j < U.n[t]; ++j) {
-      if (!wait_bar_warp(bar_addr<D>(sbase, BAR_SFULL + t), sf_ph, c)) return;
+      if (!wait_bar_warp(bar_addr(sbase, BAR_SFULL + t), sf_ph, c)) return;
       sf_ph ^= 1;
       tc_fence_after();
       uint32_t s[BN];
@@ -512,14 +592,27 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
 #pragma unroll
       for (int q = 0; q < BN / 32; ++q) reg_pin_x32(s + 32 * q);
 
-      const bool masked = tile_needs_mask(p.s, U, t, j);
-      int nvalid = 0;
-      if (masked) {
+      bool masked;
+      float m_cand;
+      if constexpr (BIAS) {
+        // Every tile adds its bias block, so every tile takes the masked form.
+        masked = true;
         int limit = U.key_len;
         if (p.s.causal) limit = min(limit, row + 1);
-        nvalid = limit - j * BN;  // keys c < nvalid of this tile are allowed
+        if (!wait_bar_warp(bar_addr(sbase, BAR_BFULL + t), bf_ph, c)) return;
+        bf_ph ^= 1;
+        m_cand = row_max_bias<BF16>(s, sl2, limit - j * BN, brow, r & 7);
+        mbar_arrive(bar_addr(sbase, BAR_BEMPTY + t));
+      } else {
+        masked = sl2 < 0.f || tile_needs_mask(p.s, U, t, j);
+        int nvalid = 0;
+        if (masked) {
+          int limit = U.key_len;
+          if (p.s.causal) limit = min(limit, row + 1);
+          nvalid = limit - j * BN;  // keys c < nvalid of this tile are allowed
+        }
+        m_cand = masked ? row_max<true>(s, sl2, nvalid) : row_max<false>(s, sl2, 0);
       }
-      const float m_cand = masked ? row_max<true>(s, sl2, nvalid) : row_max<false>(s, sl2, 0);
       // Keep the old reference max unless the new one is RESCALE_THRESHOLD
       // (log2) above it: O and l share the reference, so the result is
       // unchanged, P stays below 2^8 and the O rescale is skipped.
@@ -527,20 +620,20 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
       const float alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
       if (j > U.j0) {
         alpha_s[r] = alpha;
-        mbar_arrive(bar_addr<D>(sbase, BAR_AFULL + t));
+        mbar_arrive(bar_addr(sbase, BAR_AFULL + t));
       }
       m = m_new;
       const float mref = (m == -INFINITY) ? 0.f : m;
       const float pmax = ex2_approx(m_cand - mref);  // this tile's largest P
       const float delta = round16<BF16>(pmax) - pmax;
-      const uint32_t half_bar = bar_addr<D>(sbase, BAR_PHALF + t);
+      const uint32_t half_bar = bar_addr(sbase, BAR_PHALF + t);
       const float lsum = masked ? exp_store<BF16, true>(s, sl2, mref, t_s, half_bar)
                                 : exp_store<BF16, false>(s, sl2, mref, t_s, half_bar);
       tmem_wait_st();
       l_e = l_e * alpha + lsum;
       l_o = l_o * alpha + (lsum + delta);
       tc_fence_before();
-      mbar_arrive(bar_addr<D>(sbase, BAR_PFULL + t));
+      mbar_arrive(bar_addr(sbase, BAR_PFULL + t));
     }
     // One barrier per stats buffer: buffer (k & 1) is rewritten only after
     // the epilogue of unit k has read it (the next-but-one unit's first P·V
@@ -548,7 +641,7 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
     const int buf = units_done & 1;
     stats[(buf * 2 + t) * BM + r] = make_float4(m, l_o, l_e, 0.f);
     ++units_done;
-    mbar_arrive(bar_addr<D>(sbase, BAR_STATS + 2 * t + buf));
+    mbar_arrive(bar_addr(sbase, BAR_STATS + 2 * t + buf));
   }
 }
 
@@ -564,10 +657,10 @@ __device__ __forceinline__ uint32_t cvt2(float lo, float hi) {
   }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool BIAS>
 __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, uint32_t tmem,
                                 const Ctl& c, const CUtensorMap* tm_o) {
-  using L = Layout<D>;
+  using L = Layout<D, BIAS>;
   const int r = threadIdx.x & 127;
   const int wl = (threadIdx.x >> 5) & 3;  // warp within the group = 32-row slab
   const int lane = threadIdx.x & 31;
@@ -584,7 +677,7 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
     for (int j = U.j0 + 1; j < U.nmax && ok; ++j) {
       for (int t = 0; t < 2; ++t) {
         if (j >= U.n[t]) continue;
-        if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_AFULL + t), af_ph[t], c))) break;
+        if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_AFULL + t), af_ph[t], c))) break;
         af_ph[t] ^= 1;
         const float a = alpha_all[t * BM + r];
         if (__any_sync(0xffffffffu, a != 1.f)) {
@@ -603,7 +696,7 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
           tmem_wait_st();
         }
         tc_fence_before();
-        mbar_arrive(bar_addr<D>(sbase, BAR_OCORR + t));
+        mbar_arrive(bar_addr(sbase, BAR_OCORR + t));
       }
     }
     if (!ok) break;
@@ -616,10 +709,10 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
       const bool has = tile_active(U, t);
       if (has) {
         const int k = units_done[t]++, buf = k & 1;
-        if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_STATS + 2 * t + buf), (k >> 1) & 1, c)))
+        if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_STATS + 2 * t + buf), (k >> 1) & 1, c)))
           break;
         const float4 ml = stats[(buf * 2 + t) * BM + r];
-        if (!(ok = wait_bar_warp(bar_addr<D>(sbase, BAR_PVDONE + t), pv_ph[t], c))) break;
+        if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_PVDONE + t), pv_ph[t], c))) break;
         pv_ph[t] ^= 1;
         tc_fence_after();
         if (ml.y > 0.f) {
@@ -642,7 +735,7 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
             reg_pin_x32(o);
             if (q == D / 32 - 1) {
               tc_fence_before();
-              mbar_arrive(bar_addr<D>(sbase, BAR_OFREE + t));
+              mbar_arrive(bar_addr(sbase, BAR_OFREE + t));
             }
           } else {
 #pragma unroll
@@ -668,7 +761,7 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
           reg_pin_x32(o);
           if (q == D / 32 - 1) {
             tc_fence_before();
-            mbar_arrive(bar_addr<D>(sbase, BAR_OFREE + t));
+            mbar_arrive(bar_addr(sbase, BAR_OFREE + t));
           }
         } else {
 #pragma unroll
@@ -704,12 +797,12 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
 }
 
 // ================================================================== kernel
-template <int D, bool BF16>
+template <int D, bool BF16, bool BIAS>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                  const Params p) {
-  using L = Layout<D>;
+                  const __grid_constant__ CUtensorMap tm_b, const Params p) {
+  using L = Layout<D, BIAS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -720,22 +813,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
-      mbar_init(bar_addr<D>(sbase, BAR_QFULL + t), 1);
-      mbar_init(bar_addr<D>(sbase, BAR_QEMPTY + t), 1);
-      mbar_init(bar_addr<D>(sbase, BAR_SFULL + t), 1);
-      mbar_init(bar_addr<D>(sbase, BAR_PFULL + t), BM);
-      mbar_init(bar_addr<D>(sbase, BAR_PHALF + t), BM);
-      mbar_init(bar_addr<D>(sbase, BAR_AFULL + t), BM);
-      mbar_init(bar_addr<D>(sbase, BAR_OCORR + t), BM);
-      mbar_init(bar_addr<D>(sbase, BAR_PVDONE + t), 1);
-      mbar_init(bar_addr<D>(sbase, BAR_OFREE + t), BM);
-      mbar_init(bar_addr<D>(sbase, BAR_STATS + 2 * t), BM);
-      mbar_init(bar_addr<D>(sbase, BAR_STATS + 2 * t + 1), BM);
+      mbar_init(bar_addr(sbase, BAR_QFULL + t), 1);
+      mbar_init(bar_addr(sbase, BAR_QEMPTY + t), 1);
+      mbar_init(bar_addr(sbase, BAR_SFULL + t), 1);
+      mbar_init(bar_addr(sbase, BAR_PFULL + t), BM);
+      mbar_init(bar_addr(sbase, BAR_PHALF + t), BM);
+      mbar_init(bar_addr(sbase, BAR_AFULL + t), BM);
+      mbar_init(bar_addr(sbase, BAR_OCORR + t), BM);
+      mbar_init(bar_addr(sbase, BAR_PVDONE + t), 1);
+      mbar_init(bar_addr(sbase, BAR_OFREE + t), BM);
+      mbar_init(bar_addr(sbase, BAR_STATS + 2 * t), BM);
+      mbar_init(bar_addr(sbase, BAR_STATS + 2 * t + 1), BM);
+      mbar_init(bar_addr(sbase, BAR_BFULL + t), 1);
+      mbar_init(bar_addr(sbase, BAR_BEMPTY + t), BM);
     }
-    mbar_init(bar_addr<D>(sbase, BAR_DRAIN), 1);
+    mbar_init(bar_addr(sbase, BAR_DRAIN), 1);
     for (int s = 0; s < L::STAGES; ++s) {
-      mbar_init(bar_addr<D>(sbase, BAR_KV + s), 1);
-      mbar_init(bar_addr<D>(sbase, BAR_KV + L::STAGES + s), 1);
+      mbar_init(bar_addr(sbase, BAR_KV + s), 1);
+      mbar_init(bar_addr(sbase, BAR_KV + L::STAGES + s), 1);
     }
     *abort_flag = 0;
     mbar_init_fence();
@@ -749,6 +844,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_map(&tm_k);
     tma_prefetch_map(&tm_v);
     tma_prefetch_map(&tm_o);
+    if (BIAS) tma_prefetch_map(&tm_b);
   }
   tc_fence_before();
   __syncthreads();
@@ -759,14 +855,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // Register split: 2×176 (softmax) + 80 (correction) + 80 (MMA, loads) = 4 × 128.
   if (warp < 8) {
     setmaxnreg_inc<176>();
-    role_softmax<D, BF16>(p, smem, sbase, tmem, ctl, warp >> 2);
+    role_softmax<D, BF16, BIAS>(p, smem, sbase, tmem, ctl, warp >> 2);
   } else if (warp < 12) {
     setmaxnreg_dec<80>();
-    role_correction<D, BF16>(p, smem, sbase, tmem, ctl, &tm_o);
+    role_correction<D, BF16, BIAS>(p, smem, sbase, tmem, ctl, &tm_o);
   } else {
     setmaxnreg_dec<80>();
-    if (warp == 12) role_mma<D, BF16>(p, sbase, tmem, ctl);
-    if (warp == 13 && lane == 0) role_load<D>(p, sbase, ctl, &tm_q, &tm_k, &tm_v);
+    if (warp == 12) role_mma<D, BF16, BIAS>(p, sbase, tmem, ctl);
+    if (warp == 13 && lane == 0) role_load<D, BIAS>(p, sbase, ctl, &tm_q, &tm_k, &tm_v);
+    if constexpr (BIAS) {
+      if (warp >= 14 && lane == 0) role_bias_load<D>(p, sbase, ctl, &tm_b, warp - 14);
+    }
     __syncwarp();
   }
 
@@ -914,7 +1013,7 @@ struct DeviceInfo {
   bool init = false;
   bool sm100 = false;
   int sms = 0;
-  bool attr_set[4] = {false, false, false, false};
+  bool attr_set[8] = {false, false, false, false, false, false, false, false};
 };
 DeviceInfo g_dev[64];
 std::mutex g_dev_mu;
@@ -958,11 +1057,12 @@ int make_map(CUtensorMap* map, const void* ptr, bool bf16, int d, int n, long lo
   return FA_OK;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool BIAS = false>
 int launch(const void* q, const void* k, const void* v, void* o, const fa::Params& prm,
-           cudaStream_t stream, DeviceInfo& info, int slot, float* final_lse) {
-  using L = fa::Layout<D>;
-  auto kern = fa::fa_fwd_kernel<D, BF16>;
+           cudaStream_t stream, DeviceInfo& info, int slot, float* final_lse,
+           const void* bias = nullptr, long long bias_planes = 0) {
+  using L = fa::Layout<D, BIAS>;
+  auto kern = fa::fa_fwd_kernel<D, BF16, BIAS>;
   {
     std::lock_guard<std::mutex> lk(g_dev_mu);
     if (!info.attr_set[slot]) {
@@ -991,8 +1091,13 @@ int launch(const void* q, const void* k, const void* v, void* o, const fa::Param
                      CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
   if ((rc = make_map(&to, o, BF16, D, s.N, (long long)s.B * s.Hq, 32, 32,
                      CU_TENSOR_MAP_SWIZZLE_64B)) != FA_OK) return rc;
+  CUtensorMap tb;
+  memset(&tb, 0, sizeof(tb));
+  // bias planes [planes][N][N]: boxes of 64 keys × 128 query rows
+  if (BIAS && (rc = make_map(&tb, bias, BF16, s.N, s.N, bias_planes, 64, fa::BM,
+                             CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
   const int grid = s.num_units < info.sms ? s.num_units : info.sms;
-  kern<<<grid, fa::NUM_THREADS, L::ALLOC, stream>>>(tq, tk, tv, to, prm);
+  kern<<<grid, fa::NUM_THREADS, L::ALLOC, stream>>>(tq, tk, tv, to, tb, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
   if (prm.o_part != nullptr) {
@@ -1072,7 +1177,8 @@ int fa_unit_for(int cta, int it, int grid) { return fa::unit_for(cta, it, grid);
 namespace {
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hk,
              int N, int d, float scale, int causal, const int32_t* key_pad_lens, int splits,
-             void* workspace, size_t workspace_bytes, void* stream, int dtype) {
+             void* workspace, size_t workspace_bytes, void* stream, int dtype,
+             const void* bias = nullptr, int bias_B = 0, int bias_H = 0) {
   g_err[0] = '\0';
   // ---- arguments that need no CUDA call
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr)
@@ -1092,6 +1198,16 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (splits < 1 || splits > 16) return fail(FA_ERR_INVALID_ARG, "num_splits %d out of [1, 16]", splits);
   if ((long long)fa_num_units(B, Hq, Hk, N, causal) * splits > 0x7fffffffLL)
     return fail(FA_ERR_INVALID_ARG, "too many work units");
+  const size_t bias_bytes = bias ? (size_t)bias_B * bias_H * N * (size_t)N * 2 : 0;
+  if (bias != nullptr) {
+    if (bias_B != 1 && bias_B != B)
+      return fail(FA_ERR_INVALID_ARG, "bias batch dimension %d must be 1 or B (%d)", bias_B, B);
+    if (bias_H != 1 && bias_H != Hq)
+      return fail(FA_ERR_INVALID_ARG, "bias head dimension %d must be 1 or Hq (%d)", bias_H, Hq);
+    if (N % 8 != 0)
+      return fail(FA_ERR_UNSUPPORTED, "bias needs N %% 8 == 0 (16-byte rows), N = %d", N);
+    if (splits != 1) return fail(FA_ERR_UNSUPPORTED, "bias with split-KV is not supported");
+  }
   // ---- device and buffers
   if (!driver_fns().ok) return fail(FA_ERR_CUDA, "CUDA driver entry points unavailable");
   int dev = -1;
@@ -1128,12 +1244,23 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (overlaps(q, q_bytes) || overlaps(k, kv_bytes) || overlaps(v, kv_bytes) ||
       (lse != nullptr && overlaps(lse, (size_t)heads_q * N * 4)))
     return fail(FA_ERR_INVALID_ARG, "o overlaps an input or lse");
+  if (bias != nullptr) {
+    if ((rc = check_range("bias", bias, bias_bytes, 16)) != FA_OK) return rc;
+    if (overlaps(bias, bias_bytes)) return fail(FA_ERR_INVALID_ARG, "o overlaps bias");
+    const uintptr_t bb = reinterpret_cast<uintptr_t>(bias), be = bb + bias_bytes;
+    const uintptr_t lb = reinterpret_cast<uintptr_t>(lse);
+    if (lse != nullptr && lb < be && bb < lb + (size_t)heads_q * N * 4)
+      return fail(FA_ERR_INVALID_ARG, "lse overlaps bias");
+  }
 
   fa::Params prm;
   prm.key_pad_lens = key_pad_lens;
   prm.lse = lse;
   prm.o_part = nullptr;
   prm.lse_part = nullptr;
+  prm.bias_bmul = bias_B > 1 ? 1 : 0;
+  prm.bias_hmul = bias_H > 1 ? 1 : 0;
+  prm.bias_H = bias_H > 0 ? bias_H : 1;
   if (splits > 1) {
     const size_t need = splitkv_bytes(heads_q, N, d, splits);
     if (workspace_bytes < need)
@@ -1157,6 +1284,14 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   prm.timeout_ns = g_timeout_ns;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool bf16 = dtype == FA_BF16;
+  if (bias != nullptr) {
+    const long long planes = (long long)bias_B * bias_H;
+    if (d == 128)
+      return bf16 ? launch<128, true, true>(q, k, v, o, prm, st, info, 4, lse, bias, planes)
+                  : launch<128, false, true>(q, k, v, o, prm, st, info, 5, lse, bias, planes);
+    return bf16 ? launch<64, true, true>(q, k, v, o, prm, st, info, 6, lse, bias, planes)
+                : launch<64, false, true>(q, k, v, o, prm, st, info, 7, lse, bias, planes);
+  }
   if (d == 128)
     return bf16 ? launch<128, true>(q, k, v, o, prm, st, info, 0, lse)
                 : launch<128, false>(q, k, v, o, prm, st, info, 1, lse);
@@ -1172,6 +1307,14 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
            int dtype) {
   return fwd_impl(q, k, v, o, lse, B, Hq, Hk, N, d, scale, causal, key_pad_lens, 1, nullptr, 0,
                   stream, dtype);
+}
+
+int fa_fwd_bias(const void* q, const void* k, const void* v, const void* bias, int bias_B,
+                int bias_H, void* o, float* lse, int B, int Hq, int Hk, int N, int d, float scale,
+                int causal, const int32_t* key_pad_lens, void* stream, int dtype) {
+  if (bias == nullptr) return fail(FA_ERR_INVALID_ARG, "bias is NULL (use fa_fwd)");
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hk, N, d, scale, causal, key_pad_lens, 1, nullptr, 0,
+                  stream, dtype, bias, bias_B, bias_H);
 }
 
 size_t fa_splitkv_workspace_bytes(int B, int Hq, int N, int d, int num_splits) {
@@ -1334,6 +1477,9 @@ extern "C" int fa_fwd_splitkv_static(const void* q, const void* k, const void* v
   prm.lse = lse;
   prm.o_part = nullptr;
   prm.lse_part = nullptr;
+  prm.bias_bmul = 0;
+  prm.bias_hmul = 0;
+  prm.bias_H = 1;
   if (num_splits > 1) {
     const size_t rows = (size_t)heads_q * N * num_splits;
     prm.o_part = reinterpret_cast<float*>(scratch);

@@ -82,3 +82,15 @@ def make_inputs(w: Workload, seed: Optional[int] = None, batch_offset: int = 0):
         lens = torch.randint(lo, hi + 1, (w.B,), generator=g, dtype=torch.int32)
     return {"q": q, "k": k, "v": v, "key_pad_lens": lens}
 
+
+
+def make_bias(w: Workload, bias_B: int, bias_H: int, std: float = 2.0, seed: Optional[int] = None,
+              device: str = "cpu"):
+    """A seeded additive bias [bias_B, bias_H, N, N] in the workload's 16-bit dtype:
+    N(0, std²) samples rounded to the dtype (the workloads' pages fix no bias
+    distribution; this one moves row maxima by a few units). Drawn on
+    ``device`` with its own generator so large planes need no host copy."""
+    g = torch.Generator(device=device).manual_seed(
+        (w.seed if seed is None else seed) + 7919)
+    b = torch.randn((bias_B, bias_H, w.N, w.N), generator=g, dtype=torch.float32, device=device)
+    return b.mul_(std).to(w.torch_dtype)
