@@ -3,6 +3,7 @@
 from .attention import (  # noqa: F401
     allowed_keys,
     attention,
+    attention_backward,
     attention_key_range,
     attention_rows,
     merge_splits,

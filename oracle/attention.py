@@ -25,6 +25,11 @@ What it computes, and where the pages say so (page title, then section):
   an additive term on the scaled scores, S = scale·Q Kᵀ + bias, with bias of
   shape [Bb, Hb, N, N] broadcast over batch (Bb = 1) and heads (Hb = 1); the
   mask applies after it.
+* [NPU] (section before "实际跑一下"): standard attention keeps S and P for the
+  backward pass; the v2 FlashAttention reworks the gradient computation to
+  use less memory. No formulas are given. Read here as the gradient of the
+  forward definition above (dQ, dK, dV for a given dO), with P rebuilt from
+  Q, K and the forward's LSE instead of stored: P = exp(S − LSE).
 * [GQA] "深度探索Flash-Attention中GQA性能调优技术解析", section
   "num_splits参数的场景化配置": the attention work of one problem may be cut
   into num_splits parts. Read here as a split of the key range, each part's
@@ -54,6 +59,7 @@ __all__ = [
     "attention_key_range",
     "merge_splits",
     "split_kv_attention",
+    "attention_backward",
 ]
 
 
@@ -335,3 +341,41 @@ def split_kv_attention(q, k, v, scale, causal, key_pad_lens, bounds):
     parts = [attention_key_range(q, k, v, scale, causal, key_pad_lens, lo, hi)
              for lo, hi in zip(bounds[:-1], bounds[1:])]
     return merge_splits([p[0] for p in parts], [p[1] for p in parts])
+
+
+def attention_backward(q, k, v, o, lse, do, scale, causal=False, key_pad_lens=None):
+    """Gradients (dQ, dK, dV) of O = softmax(scale·QKᵀ + mask)·V for upstream dO.
+
+    The chain rule through the definition, row by row ([NPU] backward reading):
+    P = exp(S − LSE) with S the masked scores and LSE the forward's per-row
+    log-sum-exp (so P is the forward's softmax, rebuilt, not stored);
+    dV = Pᵀ dO; dP = dO Vᵀ; D_i = Σ_c dO_ic O_ic (= Σ_j P_ij dP_ij);
+    dS = P ⊙ (dP − D); dQ = scale · dS K; dK = scale · dSᵀ Q. A K/V head
+    shared by G query heads ([NPU] "坑四") receives the sum of their dK, dV.
+    Rows with no allowed key (LSE = −inf) have P = 0 and pass no gradient.
+    """
+    q, k, v, o, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(o), _as_f64(do)
+    lse = _as_f64(lse)
+    B, Hq, N, d = q.shape
+    Hk = k.shape[1]
+    group = Hq // Hk
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    rows = np.arange(N)
+    for b in range(B):
+        key_len = _key_len(key_pad_lens, b, N)
+        ok = allowed_keys(rows, N, causal, key_len)
+        for hq in range(Hq):
+            hk = hq // group
+            s = scores(q[b, hq], k[b, hk], scale, ok)
+            has = np.isfinite(lse[b, hq])
+            p = np.zeros((N, N))
+            p[has] = np.exp(s[has] - lse[b, hq][has][:, None])
+            dv[b, hk] += p.T @ do[b, hq]
+            dp = do[b, hq] @ v[b, hk].T
+            dsum = np.sum(do[b, hq] * o[b, hq], axis=1)
+            ds = p * (dp - dsum[:, None])
+            dq[b, hq] = scale * (ds @ k[b, hk])
+            dk[b, hk] += scale * (ds.T @ q[b, hq])
+    return dq, dk, dv

@@ -480,6 +480,93 @@ def pin_bias_broadcast_equals_repeated(orc):
         close(lrow, l0[idx], 1e-12)
 
 
+# ------------------------------------------------------- backward ([NPU] v2)
+
+def _bwd_problem(rng, B=2, Hq=4, Hk=2, N=9, d=5):
+    q, k, v, do = (rng.standard_normal(sh) for sh in
+                   [(B, Hq, N, d), (B, Hk, N, d), (B, Hk, N, d), (B, Hq, N, d)])
+    return q, k, v, do
+
+
+def pin_backward_matches_torch_autograd(orc):
+    """torch float64 math SDPA differentiated by autograd (no empty rows)."""
+    rng = np.random.default_rng(31)
+    for causal, G, lens in [(False, 1, None), (True, 2, [9, 4]), (False, 4, [3, 9]), (True, 1, None)]:
+        B, Hk, N, d = 2, 2, 9, 5
+        q, k, v, do = _bwd_problem(rng, B, Hk * G, Hk, N, d)
+        o, lse = orc.attention(q, k, v, 0.6, causal, lens)
+        dq, dk, dv = orc.attention_backward(q, k, v, o, lse, do, 0.6, causal, lens)
+        tq, tk, tv = (torch.from_numpy(x).requires_grad_() for x in (q, k, v))
+        i = torch.arange(N)[:, None]
+        j = torch.arange(N)[None, :]
+        mask = torch.stack([(j < (N if lens is None else L)) & ((j <= i) if causal else (j >= 0))
+                            for L in (lens or [N] * B)])[:, None]
+        with torch.nn.attention.sdpa_kernel(torch.nn.attention.SDPBackend.MATH):
+            out = torch.nn.functional.scaled_dot_product_attention(
+                tq, tk.repeat_interleave(G, dim=1), tv.repeat_interleave(G, dim=1),
+                attn_mask=mask, scale=0.6)
+        (out * torch.from_numpy(do)).sum().backward()
+        close(dq, tq.grad.numpy(), 1e-11)
+        close(dk, tk.grad.numpy(), 1e-11)
+        close(dv, tv.grad.numpy(), 1e-11)
+
+
+def pin_backward_finite_differences(orc):
+    """Central differences of L = Σ dO ⊙ O through the (separately pinned) forward."""
+    rng = np.random.default_rng(32)
+    q, k, v, do = _bwd_problem(rng, 1, 2, 1, 6, 3)
+    lens = [5]
+    o, lse = orc.attention(q, k, v, 0.8, True, lens)
+    grads = orc.attention_backward(q, k, v, o, lse, do, 0.8, True, lens)
+    h = 1e-6
+    for which, x in enumerate((q, k, v)):
+        for idx in [(0, 0, 0, 0), (0, 0, 3, 2), (0, x.shape[1] - 1, 5, 1), (0, 0, 2, 1)]:
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args = [q, k, v]
+            args[which] = xp
+            lp = np.sum(do * orc.attention(*args, 0.8, True, lens)[0])
+            args[which] = xm
+            lm = np.sum(do * orc.attention(*args, 0.8, True, lens)[0])
+            assert abs((lp - lm) / (2 * h) - grads[which][idx]) < 1e-7
+
+
+def pin_backward_closed_form_at_zero_scale(orc):
+    """scale = 0: P is uniform over the allowed keys, so dV_j = Σ_i dO_i / L_i over
+    the rows i that allow key j, and dQ = dK = 0."""
+    rng = np.random.default_rng(33)
+    q, k, v, do = _bwd_problem(rng, 1, 2, 2, 7, 3)
+    o, lse = orc.attention(q, k, v, 0.0, True, [5])
+    dq, dk, dv = orc.attention_backward(q, k, v, o, lse, do, 0.0, True, [5])
+    close(dq, np.zeros_like(dq), 0)
+    close(dk, np.zeros_like(dk), 0)
+    want = np.zeros_like(dv)
+    for h in range(2):
+        for i in range(7):
+            n_allowed = min(i + 1, 5)
+            for j in range(n_allowed):
+                want[0, h, j] += do[0, h, i] / n_allowed
+    close(dv, want, 1e-13)
+
+
+def pin_backward_empty_rows_and_gqa_sum(orc):
+    """A batch with no valid key passes no gradient; GQA dK, dV equal the sum
+    over the group of the gradients taken with K, V repeated per query head."""
+    rng = np.random.default_rng(34)
+    q, k, v, do = _bwd_problem(rng, 2, 4, 2, 6, 3)
+    lens = [0, 4]
+    o, lse = orc.attention(q, k, v, 0.9, False, lens)
+    dq, dk, dv = orc.attention_backward(q, k, v, o, lse, do, 0.9, False, lens)
+    assert not dq[0].any() and not dk[0].any() and not dv[0].any()
+    kr, vr = np.repeat(k, 2, axis=1), np.repeat(v, 2, axis=1)
+    o2, lse2 = orc.attention(q, kr, vr, 0.9, False, lens)
+    dq2, dk2, dv2 = orc.attention_backward(q, kr, vr, o2, lse2, do, 0.9, False, lens)
+    close(dq, dq2, 1e-13)
+    close(dk, dk2.reshape(2, 2, 2, 6, 3).sum(axis=2), 1e-13)
+    close(dv, dv2.reshape(2, 2, 2, 6, 3).sum(axis=2), 1e-13)
+
+
 def pin_hand_worked_golden(orc):
     """Problems worked by hand (tests/golden/hand_worked.json) to closed-form values."""
     for c in load_golden():

@@ -58,6 +58,13 @@ MUTATIONS = {
     "bias_head_ignored": ("hq if bias.shape[1] > 1 else 0]", "0]"),
     "bias_batch_ignored": ("b if bias.shape[0] > 1 else 0,", "0,"),
     "bias_rows_wrong_row": ("_as_f64(plane[[i]])", "_as_f64(plane[[0]])"),
+    "bwd_dsum_dropped": ("ds = p * (dp - dsum[:, None])", "ds = p * dp"),
+    "bwd_dq_unscaled": ("dq[b, hq] = scale * (ds @ k[b, hk])", "dq[b, hq] = (ds @ k[b, hk])"),
+    "bwd_dk_untransposed": ("dk[b, hk] += scale * (ds.T @ q[b, hq])", "dk[b, hk] += scale * (ds @ q[b, hq])"),
+    "bwd_dv_untransposed": ("dv[b, hk] += p.T @ do[b, hq]", "dv[b, hk] += p @ do[b, hq]"),
+    "bwd_gqa_overwrites": ("dv[b, hk] += p.T @ do[b, hq]", "dv[b, hk] = p.T @ do[b, hq]"),
+    "bwd_lse_ignored": ("np.exp(s[has] - lse[b, hq][has][:, None])", "np.exp(s[has])"),
+    "bwd_dp_wrong_v": ("dp = do[b, hq] @ v[b, hk].T", "dp = do[b, hq] @ v[b, hk][::-1].T"),
 }
 
 
