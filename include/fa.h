@@ -140,6 +140,39 @@ int fa_fwd_bias(const void* q, const void* k, const void* v, const void* bias, i
                 int bias_H, void* o, float* lse, int B, int Hq, int Hk, int N, int d, float scale,
                 int causal, const int32_t* key_pad_lens, void* stream, int dtype);
 
+/*
+ * fa_bwd — gradients of fa_fwd for an upstream gradient dout = dL/dO:
+ *     P = exp(S − LSE) (S the masked scaled scores, LSE the forward's),
+ *     dV = Pᵀ·dO,  dP = dO·Vᵀ,  D = rowsum(dO ⊙ O),  dS = P ⊙ (dP − D),
+ *     dQ = scale·dS·K,  dK = scale·dSᵀ·Q
+ * (the NPU page "FlashAttention 在昇腾 NPU 上是怎么省显存的？…" says the v2
+ * kernel reworks the backward so S and P are not stored; P is rebuilt here
+ * from Q, K and LSE). A K/V head shared by G query heads receives the sum of
+ * their dK, dV.
+ *
+ *   q, k, v, o, lse  the forward's inputs, output and LSE (o and lse exactly as
+ *                    fa_fwd wrote them), layouts as for fa_fwd.
+ *   dout             dL/dO, [B, Hq, N, d], dtype `dtype`.
+ *   dq               [B, Hq, N, d] written; dk, dv [B, Hk, N, d] written.
+ *   workspace        device pointer, 256-byte aligned, at least
+ *                    fa_bwd_workspace_bytes(B, Hq, N, d) bytes: an fp32 dQ
+ *                    accumulator and two fp32 per-row vectors. Needs no
+ *                    initialisation; scratch after the call; one per call in flight.
+ *   other arguments  as for fa_fwd (same B, Hq, Hk, N, d, scale, causal,
+ *                    key_pad_lens and dtype as the forward call).
+ * Enqueues three kernels on `stream`. dq, dk, dv and the workspace must not
+ * overlap any other argument. Returns FA_OK or a negative fa_status as fa_fwd;
+ * a device whose dynamic shared memory is not 1 KB aligned reports
+ * FA_ERR_UNSUPPORTED through fa_get_device_status().
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hk, int N, int d,
+           float scale, int causal, const int32_t* key_pad_lens, void* workspace,
+           size_t workspace_bytes, void* stream, int dtype);
+
+/* Workspace bytes fa_bwd needs (0 for invalid arguments). */
+size_t fa_bwd_workspace_bytes(int B, int Hq, int N, int d);
+
 /* Workspace bytes fa_fwd_splitkv needs: B·Hq·N·num_splits·(d + 1) floats,
  * each part rounded up to 256 bytes; 0 for num_splits == 1 and for invalid
  * arguments. */

@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["FaError", "fa_fwd", "fa_fwd_bias", "fa_fwd_splitkv", "splitkv_workspace_bytes", "load_library", "lib", "FA_OK", "FA_ERR_INVALID_ARG",
+__all__ = ["FaError", "fa_fwd", "fa_bwd", "fa_fwd_bias", "fa_fwd_splitkv", "splitkv_workspace_bytes", "load_library", "lib", "FA_OK", "FA_ERR_INVALID_ARG",
            "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT"]
 
 FA_OK = 0
@@ -43,6 +43,11 @@ def load_library(path=LIB_PATH):
     L.fa_fwd.argtypes = [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                          c_int, c_int, c_float, c_int, c_void_p, c_void_p, c_int]
     L.fa_fwd.restype = c_int
+    L.fa_bwd.argtypes = [c_void_p] * 9 + [c_int] * 5 + [c_float, c_int, c_void_p, c_void_p,
+                                                       ctypes.c_size_t, c_void_p, c_int]
+    L.fa_bwd.restype = c_int
+    L.fa_bwd_workspace_bytes.argtypes = [c_int] * 4
+    L.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
     L.fa_fwd_bias.argtypes = [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p,
                               c_void_p, c_int, c_int, c_int, c_int, c_int, c_float, c_int,
                               c_void_p, c_void_p, c_int]
@@ -159,6 +164,37 @@ def fa_fwd_bias(q, k, v, bias, causal=False, scale=None, key_pad_lens=None, out=
                               key_pad_lens.data_ptr() if key_pad_lens is not None else None,
                               stream, _DTYPES[q.dtype]))
     return (out, lse) if return_lse else out
+
+
+def fa_bwd(q, k, v, o, lse, dout, causal=False, scale=None, key_pad_lens=None, dq=None, dk=None,
+           dv=None, workspace=None, stream=None):
+    """(dq, dk, dv) of the attention forward for upstream gradient ``dout``.
+
+    ``o`` and ``lse`` are the forward's outputs for the same q, k, v, causal,
+    scale and key_pad_lens. The fp32 workspace is allocated here when None.
+    """
+    (B, Hq, Hk, N, d), _, _, scale, stream = _prepare(q, k, v, key_pad_lens, o, lse, True,
+                                                      scale, stream)
+    for name, t in (("o", o), ("dout", dout)):
+        if not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, Hq, N, d) or \
+                t.dtype != q.dtype:
+            raise FaError(FA_ERR_INVALID_ARG, f"{name} must be a contiguous CUDA tensor like q")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, N) or not lse.is_contiguous():
+        raise FaError(FA_ERR_INVALID_ARG, "lse must be a contiguous float32 [B, Hq, N] tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = lib.fa_bwd_workspace_bytes(B, Hq, N, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        check(lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                         dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hk,
+                         N, d, scale, 1 if causal else 0,
+                         key_pad_lens.data_ptr() if key_pad_lens is not None else None,
+                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                         stream, _DTYPES[q.dtype]))
+    return dq, dk, dv
 
 
 def splitkv_workspace_bytes(B, Hq, N, d, num_splits):

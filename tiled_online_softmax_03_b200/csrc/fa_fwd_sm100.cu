@@ -960,6 +960,8 @@ __global__ void fa_exp2_selftest_kernel(const float* x, float* y_fma, float* y_m
   }
 }
 
+#include "fa_bwd_sm100.cuh"
+
 }  // namespace fa
 
 // ==================================================================== host
@@ -1014,6 +1016,7 @@ struct DeviceInfo {
   bool sm100 = false;
   int sms = 0;
   bool attr_set[8] = {false, false, false, false, false, false, false, false};
+  bool bwd_attr_set[4] = {false, false, false, false};
 };
 DeviceInfo g_dev[64];
 std::mutex g_dev_mu;
@@ -1496,4 +1499,169 @@ extern "C" int fa_fwd_splitkv_static(const void* q, const void* k, const void* v
                 : launch<128, false>(q, k, v, o, prm, st, info, 1, lse);
   return bf16 ? launch<64, true>(q, k, v, o, prm, st, info, 2, lse)
               : launch<64, false>(q, k, v, o, prm, st, info, 3, lse);
+}
+
+// ================================================================ backward
+namespace {
+struct BwdWs {
+  size_t dq_off, lse2_off, dsum_off, bytes;
+};
+BwdWs bwd_ws(long long heads_q, int N, int d) {
+  const size_t npad = (size_t)(N + 127) / 128 * 128;
+  BwdWs w;
+  w.dq_off = 0;
+  w.lse2_off = ((size_t)heads_q * N * d * 4 + 255) / 256 * 256;
+  w.dsum_off = w.lse2_off + ((size_t)heads_q * npad * 4 + 255) / 256 * 256;
+  w.bytes = w.dsum_off + ((size_t)heads_q * npad * 4 + 255) / 256 * 256;
+  return w;
+}
+
+template <int D, bool BF16>
+int bwd_launch(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dout, void* dq, void* dk, void* dv, const fa::bwd::BParams& bp,
+               float* dqacc, float* lse2, float* dsum, cudaStream_t st, DeviceInfo& info, int slot) {
+  using L = fa::bwd::BLayout<D>;
+  auto kern = fa::bwd::fa_bwd_kernel<D, BF16>;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!info.bwd_attr_set[slot]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES) !=
+          cudaSuccess)
+        return fail(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
+      info.bwd_attr_set[slot] = true;
+    }
+  }
+  const long long BH = (long long)bp.B * bp.Hq;
+  CUtensorMap tq, tk, tv, tdo;
+  int rc;
+  if ((rc = make_map(&tq, q, BF16, D, bp.N, BH, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
+  if ((rc = make_map(&tk, k, BF16, D, bp.N, (long long)bp.B * bp.Hk, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
+  if ((rc = make_map(&tv, v, BF16, D, bp.N, (long long)bp.B * bp.Hk, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
+  if ((rc = make_map(&tdo, dout, BF16, D, bp.N, BH, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+    return rc;
+  const long long pre_rows = BH * bp.Npad;
+  long long pre_blocks = (pre_rows + 7) / 8;
+  if (pre_blocks > (long long)info.sms * 32) pre_blocks = (long long)info.sms * 32;
+  fa::bwd::fa_bwd_pre_kernel<D, BF16><<<(unsigned)pre_blocks, 256, 0, st>>>(
+      o, dout, lse, lse2, dsum, dqacc, BH, bp.N, bp.Npad);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "backward prologue launch: %s", cudaGetErrorString(e));
+  const int grid = bp.num_units < info.sms ? bp.num_units : info.sms;
+  kern<<<grid, fa::bwd::NUM_THREADS, L::BYTES, st>>>(tq, tk, tv, tdo, bp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
+  const long long n8 = BH * bp.N * D / 8;
+  long long post_blocks = (n8 + 255) / 256;
+  if (post_blocks > (long long)info.sms * 32) post_blocks = (long long)info.sms * 32;
+  fa::bwd::fa_bwd_post_kernel<BF16><<<(unsigned)post_blocks, 256, 0, st>>>(dqacc, dq, bp.scale, n8);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "backward epilogue launch: %s", cudaGetErrorString(e));
+  return FA_OK;
+}
+}  // namespace
+
+extern "C" size_t fa_bwd_workspace_bytes(int B, int Hq, int N, int d) {
+  if (B < 1 || Hq < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  return bwd_ws((long long)B * Hq, N, d).bytes;
+}
+
+extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                      const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hk, int N,
+                      int d, float scale, int causal, const int32_t* key_pad_lens, void* workspace,
+                      size_t workspace_bytes, void* stream, int dtype) {
+  g_err[0] = '\0';
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr ||
+      dout == nullptr || dq == nullptr || dk == nullptr || dv == nullptr)
+    return fail(FA_ERR_INVALID_ARG, "q, k, v, o, lse, dout, dq, dk and dv must be non-NULL");
+  if (B < 1 || Hq < 1 || Hk < 1 || N < 1)
+    return fail(FA_ERR_INVALID_ARG, "B, Hq, Hk and N must be >= 1");
+  if (Hq % Hk != 0) return fail(FA_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hk (%d)", Hq, Hk);
+  if (d != 64 && d != 128)
+    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", d);
+  if (dtype != FA_FP16 && dtype != FA_BF16) return fail(FA_ERR_UNSUPPORTED, "unknown dtype %d", dtype);
+  if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "scale must be finite");
+  if (causal != 0 && causal != 1) return fail(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  const long long heads_q = (long long)B * Hq, heads_k = (long long)B * Hk;
+  if (heads_q > 0x7fffffffLL || N > (1 << 30))
+    return fail(FA_ERR_INVALID_ARG, "problem too large for 32-bit tile coordinates");
+  const long long units = heads_k * ((N + 127) / 128);
+  if (units > 0x7fffffffLL) return fail(FA_ERR_INVALID_ARG, "too many work units");
+  const BwdWs ws = bwd_ws(heads_q, N, d);
+  if (workspace_bytes < ws.bytes)
+    return fail(FA_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", workspace_bytes, ws.bytes);
+  // ---- device and buffers
+  if (!driver_fns().ok) return fail(FA_ERR_CUDA, "CUDA driver entry points unavailable");
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return fail(FA_ERR_CUDA, "no current CUDA device");
+  DeviceInfo& info = g_dev[dev];
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!info.init) {
+      cudaDeviceProp prop;
+      if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess)
+        return fail(FA_ERR_CUDA, "cudaGetDeviceProperties failed");
+      info.sm100 = prop.major == 10 && prop.minor == 0;
+      info.sms = prop.multiProcessorCount;
+      info.init = true;
+    }
+  }
+  if (!info.sm100) return fail(FA_ERR_UNSUPPORTED, "device %d is not sm_100", dev);
+  const size_t q_bytes = (size_t)heads_q * N * d * 2, kv_bytes = (size_t)heads_k * N * d * 2;
+  const size_t lse_bytes = (size_t)heads_q * N * 4;
+  int rc;
+  if ((rc = check_range("q", q, q_bytes, 16)) != FA_OK) return rc;
+  if ((rc = check_range("k", k, kv_bytes, 16)) != FA_OK) return rc;
+  if ((rc = check_range("v", v, kv_bytes, 16)) != FA_OK) return rc;
+  if ((rc = check_range("o", o, q_bytes, 16)) != FA_OK) return rc;
+  if ((rc = check_range("lse", lse, lse_bytes, 4)) != FA_OK) return rc;
+  if ((rc = check_range("dout", dout, q_bytes, 16)) != FA_OK) return rc;
+  if ((rc = check_range("dq", dq, q_bytes, 16)) != FA_OK) return rc;
+  if ((rc = check_range("dk", dk, kv_bytes, 16)) != FA_OK) return rc;
+  if ((rc = check_range("dv", dv, kv_bytes, 16)) != FA_OK) return rc;
+  if ((rc = check_range("workspace", workspace, ws.bytes, 256)) != FA_OK) return rc;
+  if (key_pad_lens != nullptr &&
+      (rc = check_range("key_pad_lens", key_pad_lens, (size_t)B * 4, 4)) != FA_OK)
+    return rc;
+  // outputs and the workspace may overlap nothing else
+  struct Span { const void* p; size_t n; };
+  const Span outs[4] = {{dq, q_bytes}, {dk, kv_bytes}, {dv, kv_bytes}, {workspace, ws.bytes}};
+  const Span all[10] = {{q, q_bytes}, {k, kv_bytes}, {v, kv_bytes}, {o, q_bytes}, {lse, lse_bytes},
+                        {dout, q_bytes}, {dq, q_bytes}, {dk, kv_bytes}, {dv, kv_bytes},
+                        {workspace, ws.bytes}};
+  for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < 10; ++j) {
+      if (outs[i].p == all[j].p && outs[i].n == all[j].n && (j == 6 + i)) continue;  // itself
+      const uintptr_t a = reinterpret_cast<uintptr_t>(outs[i].p), b = reinterpret_cast<uintptr_t>(all[j].p);
+      if (a < b + all[j].n && b < a + outs[i].n)
+        return fail(FA_ERR_INVALID_ARG, "an output or the workspace overlaps another argument");
+    }
+  fa::bwd::BParams bp;
+  bp.B = B; bp.Hq = Hq; bp.Hk = Hk; bp.N = N; bp.G = Hq / Hk;
+  bp.NM = (N + 127) / 128;
+  bp.Npad = bp.NM * 128;
+  bp.causal = causal;
+  bp.num_units = (int)units;
+  bp.key_pad_lens = key_pad_lens;
+  uint8_t* wsb = reinterpret_cast<uint8_t*>(workspace);
+  float* dqacc = reinterpret_cast<float*>(wsb + ws.dq_off);
+  float* lse2 = reinterpret_cast<float*>(wsb + ws.lse2_off);
+  float* dsum = reinterpret_cast<float*>(wsb + ws.dsum_off);
+  bp.lse2 = lse2;
+  bp.dsum = dsum;
+  bp.dqacc = dqacc;
+  bp.dk = dk;
+  bp.dv = dv;
+  bp.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  bp.scale = scale;
+  bp.timeout_ns = g_timeout_ns;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == FA_BF16;
+  if (d == 128)
+    return bf16 ? bwd_launch<128, true>(q, k, v, o, lse, dout, dq, dk, dv, bp, dqacc, lse2, dsum, st, info, 0)
+                : bwd_launch<128, false>(q, k, v, o, lse, dout, dq, dk, dv, bp, dqacc, lse2, dsum, st, info, 1);
+  return bf16 ? bwd_launch<64, true>(q, k, v, o, lse, dout, dq, dk, dv, bp, dqacc, lse2, dsum, st, info, 2)
+              : bwd_launch<64, false>(q, k, v, o, lse, dout, dq, dk, dv, bp, dqacc, lse2, dsum, st, info, 3);
 }
