@@ -546,8 +546,9 @@ __device__ __forceinline__ float exp_store(const uint32_t (&s)[BN], float sl2, f
       tc_fence_before();
       mbar_arrive(half_bar);
     }
+    if (i == 3 * BN / 8 - 1) tmem_st_x16(t_p + 32, pk + 32);
   }
-  tmem_st_x32(t_p + 32, pk + 32);
+  tmem_st_x16(t_p + 48, pk + 48);
   const uint64_t e2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
   return f2_lo(e2) + f2_hi(e2);
 }
@@ -617,18 +618,19 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
       // (log2) above it: O and l share the reference, so the result is
       // unchanged, P stays below 2^8 and the O rescale is skipped.
       const float m_new = (m_cand > m + RESCALE_THRESHOLD) ? m_cand : m;
-      const float alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
+      float alpha = 1.f;
+      if (m_new != m) alpha = ex2_approx(m - m_new);
       if (j > U.j0) {
         alpha_s[r] = alpha;
         mbar_arrive(bar_addr(sbase, BAR_AFULL + t));
       }
       m = m_new;
       const float mref = (m == -INFINITY) ? 0.f : m;
-      const float pmax = ex2_approx(m_cand - mref);  // this tile's largest P
-      const float delta = round16<BF16>(pmax) - pmax;
       const uint32_t half_bar = bar_addr(sbase, BAR_PHALF + t);
       const float lsum = masked ? exp_store<BF16, true>(s, sl2, mref, t_s, half_bar)
                                 : exp_store<BF16, false>(s, sl2, mref, t_s, half_bar);
+      const float pmax = ex2_approx(m_cand - mref);  // this tile's largest P
+      const float delta = round16<BF16>(pmax) - pmax;
       tmem_wait_st();
       l_e = l_e * alpha + lsum;
       l_o = l_o * alpha + (lsum + delta);
