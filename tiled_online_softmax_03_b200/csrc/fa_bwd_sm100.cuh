@@ -25,7 +25,9 @@
 //   MMA warp      dV += Pᵀ·dO, dK += dSᵀ·Q (A from TMEM), dQ_part = dS·K
 //                 (A = dSᵀ read MN-major from shared memory) into the dPᵀ
 //                 columns
-//   drain warps   thread = query row: dQ_part from TMEM, red.global.add.v4
+//   drain warps   thread = query row: dQ_part from TMEM into the dSᵀ tile
+//                 (free once the dQ MMA has read it) as 32-column fp32 boxes,
+//                 added into the fp32 dQ buffer by TMA reduce-add
 // TMEM columns: Sᵀ/Pᵀ [0,128), dPᵀ/dSᵀ/dQ_part [128,256), dV and dK after.
 
 namespace bwd {
@@ -47,7 +49,8 @@ enum {
   BB_ACC_FULL = 10, // MMA -> drain: the unit's dK, dV complete
   BB_ACC_FREE = 11, // drain -> MMA: dK, dV read
   BB_DRAIN = 12,    // MMA drain on the abort path
-  BB_COUNT = 13
+  BB_STG_FREE = 13, // drain -> softmax: the dSᵀ tile, used as dQ staging, read by TMA
+  BB_COUNT = 14
 };
 
 // Shared memory, no slack: the tiles need a 1 KB-aligned base, which the
@@ -269,6 +272,8 @@ __device__ void bwd_softmax(const BParams& p, uint8_t* smem, uint32_t sbase, uin
       if (!wait_bar_warp(bbar(sbase, BB_QD_FULL + stg), use & 1, c)) return;
       if (!wait_bar_warp(bbar(sbase, BB_SDP_FULL), step_ct & 1, c)) return;
       tc_fence_after();
+      // the dSᵀ tile doubles as the drain's dQ staging: wait until TMA has read it
+      if (step_ct > 0 && !wait_bar_warp(bbar(sbase, BB_STG_FREE), (step_ct - 1) & 1, c)) return;
       const int m = U.m_lo + s % U.nm;
       const float* lse2 = reinterpret_cast<const float*>(smem + L::OFF_LD + stg * 1024);
       const float* dsum = lse2 + 128;
@@ -319,19 +324,26 @@ __device__ void bwd_softmax(const BParams& p, uint8_t* smem, uint32_t sbase, uin
 
 // --------------------------------------------------- dQ drain and dK/dV out
 template <int D, bool BF16>
-__device__ void bwd_drain(const BParams& p, uint32_t sbase, uint32_t tmem, const Ctl& c) {
+__device__ void bwd_drain(const BParams& p, uint8_t* smem, uint32_t sbase, uint32_t tmem,
+                          const Ctl& c, const CUtensorMap* tm_dq) {
+  using L = BLayout<D>;
   const int r = threadIdx.x & 127;  // TMEM lane: query row (dQ_part), key row (dK, dV)
   const uint32_t lane_base = (uint32_t)((threadIdx.x >> 5) & 3) * 32;
   const uint32_t t_row = tmem + (lane_base << 16);
+  const int lane = threadIdx.x & 31, wl = (threadIdx.x >> 5) & 3;
+  constexpr int STG_BOX = BQ * 32 * 4;  // one [128 rows][32 fp32] staging box, 16 KB
   int step_ct = 0, acc_units = 0;
   BUnit U;
   for (int it = 0; bwd_unit(p, it, U); ++it) {
     for (int s = 0; s < U.steps; ++s, ++step_ct) {
-      if (!wait_bar_warp(bbar(sbase, BB_DQ_FULL), step_ct & 1, c)) return;
+      if (!wait_bar_warp(bbar(sbase, BB_DQ_FULL), step_ct & 1, c)) goto done;
       tc_fence_after();
       const int hq = U.hk * p.G + s / U.nm, m = U.m_lo + s % U.nm;
-      const int q = m * BQ + r;
-      float* dst = p.dqacc + ((size_t)(U.b * p.Hq + hq) * p.N + q) * D;
+      const int head = U.b * p.Hq + hq;
+      // dQ_part through the 32 KB dSᵀ tile: two staging boxes of [128 rows][32
+      // fp32]; each warp stages its own 32 rows and its lane 0 adds that 4 KB
+      // slab into dQ by TMA (no cross-warp barrier). Row r, 16-byte chunk i
+      // sits at chunk i ^ (r & 7) of its 128-byte row (128-byte swizzle).
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t v[32];
@@ -342,20 +354,35 @@ __device__ void bwd_drain(const BParams& p, uint32_t sbase, uint32_t tmem, const
           tc_fence_before();
           mbar_arrive(bbar(sbase, BB_DQ_FREE));
         }
-        if (q < p.N) {
+        if (cc >= 2) {  // this box was staged two chunks ago: has TMA read it?
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+        }
+        const uint32_t slab = L::OFF_DS + (cc & 1) * STG_BOX + wl * 32 * 128;
+        uint8_t* row = smem + slab + (r & 31) * 128;
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            red_add_v4(dst + 32 * cc + 4 * i, __uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                       __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        for (int i = 0; i < 8; ++i)
+          *reinterpret_cast<uint4*>(row + ((i ^ (r & 7)) << 4)) =
+              make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(tm_dq, sbase + slab, 32 * cc, m * BQ + wl * 32, head);
+          bulk_commit_group();
         }
       }
+      if (lane == 0) {
+        bulk_wait_group_read<0>();
+        mbar_arrive(bbar(sbase, BB_STG_FREE));
+      }
+      __syncwarp();
     }
     // ---- the unit's dK (×scale) and dV rows
     const int key = U.n * BK + r;
     const size_t orow = ((size_t)(U.b * p.Hk + U.hk) * p.N + key) * D;
     const bool has = U.steps > 0;
     if (has) {
-      if (!wait_bar_warp(bbar(sbase, BB_ACC_FULL), acc_units & 1, c)) return;
+      if (!wait_bar_warp(bbar(sbase, BB_ACC_FULL), acc_units & 1, c)) goto done;
       tc_fence_after();
     }
 #pragma unroll 1
@@ -392,13 +419,17 @@ __device__ void bwd_drain(const BParams& p, uint32_t sbase, uint32_t tmem, const
     }
     if (has) ++acc_units;
   }
+done:
+  // the TMA reductions into dQ complete before the CTA may exit
+  if (lane == 0) bulk_wait_group<0>();
+  __syncwarp();
 }
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const BParams p) {
+                  const __grid_constant__ CUtensorMap tm_dq, const BParams p) {
   using L = BLayout<D>;
   extern __shared__ __align__(1024) uint8_t bsmem[];
   const uint32_t sbase = smem_addr(bsmem);
@@ -423,6 +454,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(bbar(sbase, BB_ACC_FULL), 1);
     mbar_init(bbar(sbase, BB_ACC_FREE), 128);
     mbar_init(bbar(sbase, BB_DRAIN), 1);
+    mbar_init(bbar(sbase, BB_STG_FREE), 4);  // lane 0 of each drain warp
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -435,6 +467,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_map(&tm_k);
     tma_prefetch_map(&tm_v);
     tma_prefetch_map(&tm_do);
+    tma_prefetch_map(&tm_dq);
   }
   tc_fence_before();
   __syncthreads();
@@ -444,7 +477,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp < 4) {
     bwd_softmax<D, BF16>(p, bsmem, sbase, tmem, ctl);
   } else if (warp < 8) {
-    bwd_drain<D, BF16>(p, sbase, tmem, ctl);
+    bwd_drain<D, BF16>(p, bsmem, sbase, tmem, ctl, &tm_dq);
   } else {
     if (warp == 8) bwd_mma<D, BF16>(p, sbase, tmem, ctl);
     if (warp == 9 && lane == 0) bwd_load<D>(p, sbase, ctl, &tm_q, &tm_k, &tm_v, &tm_do);

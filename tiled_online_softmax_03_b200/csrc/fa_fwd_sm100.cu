@@ -1543,6 +1543,19 @@ int bwd_launch(const void* q, const void* k, const void* v, const void* o, const
                      CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
   if ((rc = make_map(&tdo, dout, BF16, D, bp.N, BH, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
     return rc;
+  // fp32 dQ accumulator [B·Hq][N][D], reduced into in 32-column × 32-row boxes
+  CUtensorMap tdq;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)bp.N, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)D * 4 * (cuuint64_t)bp.N};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = driver_fns().encode(&tdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dqacc, dims, strides,
+                                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled (dQ) failed (%d)", (int)r);
+  }
   const long long pre_rows = BH * bp.Npad;
   long long pre_blocks = (pre_rows + 7) / 8;
   if (pre_blocks > (long long)info.sms * 32) pre_blocks = (long long)info.sms * 32;
@@ -1551,7 +1564,7 @@ int bwd_launch(const void* q, const void* k, const void* v, const void* o, const
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "backward prologue launch: %s", cudaGetErrorString(e));
   const int grid = bp.num_units < info.sms ? bp.num_units : info.sms;
-  kern<<<grid, fa::bwd::NUM_THREADS, L::BYTES, st>>>(tq, tk, tv, tdo, bp);
+  kern<<<grid, fa::bwd::NUM_THREADS, L::BYTES, st>>>(tq, tk, tv, tdo, tdq, bp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
   const long long n8 = BH * bp.N * D / 8;

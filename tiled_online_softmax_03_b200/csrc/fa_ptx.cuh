@@ -93,6 +93,19 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                "f"(c), "f"(d)
                : "memory");
 }
+// 3-D tiled reduce-add shared -> global (f32 add into the tensor; rows past
+// the extent are clipped).
+__device__ __forceinline__ void tma_reduce_add_3d(const void* map, uint32_t src, int c0, int c1,
+                                                  int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+      ::"l"(map), "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+// Barrier over the `count` threads of a warp group that use named barrier `id`.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
