@@ -18,30 +18,34 @@
 //
 // Per step (Q, dO, LSE·log2e and D of query tile m staged by TMA, two stages):
 //   MMA warp      Sᵀ = K·Qᵀ and dPᵀ = V·dOᵀ into TMEM (keys are the M rows)
-//   softmax warps thread k = key row: Pᵀ = exp2(Sᵀ·scale·log2e − LSE·log2e)
-//                 (masked keys → 0), dSᵀ = Pᵀ ⊙ (dPᵀ − D); Pᵀ and dSᵀ go to
-//                 TMEM as 16-bit pairs over Sᵀ and dPᵀ, dSᵀ also to shared
-//                 memory in the 128-byte-swizzled layout of an MN-major operand
+//   softmax warps (eight: thread = key row, warps 0-3 queries 0-63 of the
+//                 tile, warps 4-7 queries 64-127): Pᵀ = exp2(Sᵀ·scale·log2e −
+//                 LSE·log2e) (masked keys → 0), dSᵀ = Pᵀ ⊙ (dPᵀ − D); Pᵀ and dSᵀ
+//                 go to TMEM as 16-bit pairs over Sᵀ and dPᵀ, then dSᵀ (read back
+//                 from TMEM) to shared memory in the 128-byte-swizzled layout
+//                 of an MN-major operand
 //   MMA warp      dV += Pᵀ·dO, dK += dSᵀ·Q (A from TMEM), dQ_part = dS·K
 //                 (A = dSᵀ read MN-major from shared memory) into the dPᵀ
 //                 columns
 //   drain warps   thread = query row: dQ_part from TMEM into the dSᵀ tile
 //                 (free once the dQ MMA has read it) as 32-column fp32 boxes,
 //                 added into the fp32 dQ buffer by TMA reduce-add
-// TMEM columns: Sᵀ/Pᵀ [0,128), dPᵀ/dSᵀ/dQ_part [128,256), dV and dK after.
+// TMEM columns: Sᵀ/Pᵀ [0,128), dPᵀ/dSᵀ/dQ_part [128,256), dV and dK after;
+// the 16-bit pairs of queries 64·h + [0, 64) occupy columns 64·h + [0, 32)
+// of the Sᵀ and dPᵀ ranges.
 
 namespace bwd {
 
 constexpr int BK = 128;  // keys per unit
 constexpr int BQ = 128;  // queries per step
-constexpr int NUM_THREADS = 384;
+constexpr int NUM_THREADS = 512;
 constexpr int TMEM_COLS = 512;
 
 enum {
   BB_KV_FULL = 0,   // TMA -> MMA: K and V of the unit loaded
   BB_KV_EMPTY = 1,  // MMA -> TMA: the unit's MMAs no longer read K, V
   BB_QD_FULL = 2,   // [2] TMA -> MMA, softmax: Q, dO, LSE·log2e, D of a step
-  BB_QD_EMPTY = 4,  // [2] MMA (commit) + 4 softmax warps -> TMA: stage read
+  BB_QD_EMPTY = 4,  // [2] MMA (commit) + 8 softmax warps -> TMA: stage read
   BB_SDP_FULL = 6,  // MMA -> softmax: Sᵀ and dPᵀ in TMEM
   BB_P_READY = 7,   // softmax -> MMA: Pᵀ, dSᵀ in TMEM and dSᵀ in smem
   BB_DQ_FULL = 8,   // MMA -> drain: dQ_part in TMEM
@@ -193,12 +197,14 @@ __device__ void bwd_mma(const BParams& p, uint32_t sbase, uint32_t tmem, const C
       umma_ss_warp(d_t, a + off, b + off, ID_S, 1u);
     }
   };
-  // C[128][D] (+)= A(TMEM, 16-bit pairs)[128][128]·B[128][D], B MN-major
+  // C[128][D] (+)= A(TMEM, 16-bit pairs)[128][128]·B[128][D], B MN-major. The
+  // pairs of queries 64·h + [0, 64) sit in columns 64·h + [0, 32) (the softmax
+  // halves' layout), so K step k (16 queries) reads columns 64·(k/4) + 8·(k%4).
   auto mma_tk = [&](uint32_t d_t, uint32_t a_t, uint64_t b, uint32_t acc) {
     umma_ts_warp(d_t, a_t, b, ID_G, acc);
 #pragma unroll
     for (int k = 1; k < BQ / 16; ++k)
-      umma_ts_warp(d_t, a_t + k * 8, b + ((k * 16 * 128) >> 4), ID_G, 1u);
+      umma_ts_warp(d_t, a_t + (k >> 2) * 64 + (k & 3) * 8, b + ((k * 16 * 128) >> 4), ID_G, 1u);
   };
   int units = 0, acc_units = 0, step_ct = 0;
   bool ok = true;
@@ -256,10 +262,11 @@ template <int D, bool BF16>
 __device__ void bwd_softmax(const BParams& p, uint8_t* smem, uint32_t sbase, uint32_t tmem,
                             const Ctl& c) {
   using L = BLayout<D>;
-  const int k = threadIdx.x & 127;  // key row of the block = TMEM lane
+  const int k = threadIdx.x & 127;       // key row of the block = TMEM lane
+  const int half = (threadIdx.x >> 7) & 1;  // queries [64·half, 64·half + 64) of the tile
   const uint32_t lane_base = (uint32_t)((threadIdx.x >> 5) & 3) * 32;
   const uint32_t t_s = tmem + (lane_base << 16), t_dp = t_s + 128;
-  uint8_t* ds_row = smem + L::OFF_DS + k * 128;
+  uint8_t* ds_row = smem + L::OFF_DS + half * SW128_BOX_BYTES + k * 128;
   const int sw = k & 7;
   int step_ct = 0;
   BUnit U;
@@ -272,15 +279,14 @@ __device__ void bwd_softmax(const BParams& p, uint8_t* smem, uint32_t sbase, uin
       if (!wait_bar_warp(bbar(sbase, BB_QD_FULL + stg), use & 1, c)) return;
       if (!wait_bar_warp(bbar(sbase, BB_SDP_FULL), step_ct & 1, c)) return;
       tc_fence_after();
-      // the dSᵀ tile doubles as the drain's dQ staging: wait until TMA has read it
-      if (step_ct > 0 && !wait_bar_warp(bbar(sbase, BB_STG_FREE), (step_ct - 1) & 1, c)) return;
       const int m = U.m_lo + s % U.nm;
       const float* lse2 = reinterpret_cast<const float*>(smem + L::OFF_LD + stg * 1024);
       const float* dsum = lse2 + 128;
       // queries j of the tile with key <= m·128 + j (causal), all if not causal
       const int q_first = p.causal ? key - m * BQ : 0;
 #pragma unroll 1
-      for (int cc = 0; cc < BQ / 32; ++cc) {
+      for (int cq = 0; cq < 2; ++cq) {
+        const int cc = 2 * half + cq;  // 32-query chunk of the tile
         uint32_t sv[32], dp[32];
         tmem_ld_x32(t_s + 32 * cc, sv);
         tmem_ld_x32(t_dp + 32 * cc, dp);
@@ -302,17 +308,24 @@ __device__ void bwd_softmax(const BParams& p, uint8_t* smem, uint32_t sbase, uin
           pk[i] = round_pack<BF16>(pv[0], pv[1]);
           dk2[i] = round_pack<BF16>(dv[0], dv[1]);
         }
-        tmem_st_x16(t_s + 16 * cc, pk);
-        tmem_st_x16(t_dp + 16 * cc, dk2);
-        // dSᵀ row k, queries 32·cc .. +31: four 16-byte chunks of box cc/2,
-        // chunk index ((cc & 1)·4 + i) stored at that index ^ (k & 7)
-        uint8_t* box = ds_row + (cc >> 1) * SW128_BOX_BYTES;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          *reinterpret_cast<uint4*>(box + ((((cc & 1) * 4 + i) ^ sw) << 4)) =
-              make_uint4(dk2[4 * i], dk2[4 * i + 1], dk2[4 * i + 2], dk2[4 * i + 3]);
+        // packed pairs of half h go to columns 64·h + [0, 32): only columns this
+        // thread has already read, never the other half's unread ones
+        tmem_st_x16(t_s + 64 * half + 16 * cq, pk);
+        tmem_st_x16(t_dp + 64 * half + 16 * cq, dk2);
       }
       tmem_wait_st();
+      // dSᵀ to the shared tile (it doubles as the drain's dQ staging: wait until
+      // TMA has read that): this thread's 64 queries are one 128-byte row of box
+      // `half`, 16-byte chunk i stored at chunk i ^ (k & 7)
+      if (step_ct > 0 && !wait_bar_warp(bbar(sbase, BB_STG_FREE), (step_ct - 1) & 1, c)) return;
+      uint32_t w[32];
+      tmem_ld_x32(t_dp + 64 * half, w);
+      tmem_wait_ld();
+      reg_pin_x32(w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        *reinterpret_cast<uint4*>(ds_row + ((i ^ sw) << 4)) =
+            make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       fence_proxy_async_smem();  // generic-proxy writes of dSᵀ, read by the MMA
       tc_fence_before();
       mbar_arrive(bbar(sbase, BB_P_READY));
@@ -445,10 +458,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(bbar(sbase, BB_KV_EMPTY), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bbar(sbase, BB_QD_FULL + s), 1);
-      mbar_init(bbar(sbase, BB_QD_EMPTY + s), 1 + 4);  // MMA commit + one per softmax warp
+      mbar_init(bbar(sbase, BB_QD_EMPTY + s), 1 + 8);  // MMA commit + one per softmax warp
     }
     mbar_init(bbar(sbase, BB_SDP_FULL), 1);
-    mbar_init(bbar(sbase, BB_P_READY), 128);
+    mbar_init(bbar(sbase, BB_P_READY), 256);
     mbar_init(bbar(sbase, BB_DQ_FULL), 1);
     mbar_init(bbar(sbase, BB_DQ_FREE), 128);
     mbar_init(bbar(sbase, BB_ACC_FULL), 1);
@@ -458,11 +471,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     *abort_flag = 0;
     mbar_init_fence();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 9 && lane == 0) {
+  if (warp == 13 && lane == 0) {
     tma_prefetch_map(&tm_q);
     tma_prefetch_map(&tm_k);
     tma_prefetch_map(&tm_v);
@@ -474,18 +487,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Ctl ctl{abort_flag, p.timeout_ns};
-  if (warp < 4) {
+  if (warp < 8) {
     bwd_softmax<D, BF16>(p, bsmem, sbase, tmem, ctl);
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     bwd_drain<D, BF16>(p, bsmem, sbase, tmem, ctl, &tm_dq);
   } else {
-    if (warp == 8) bwd_mma<D, BF16>(p, sbase, tmem, ctl);
-    if (warp == 9 && lane == 0) bwd_load<D>(p, sbase, ctl, &tm_q, &tm_k, &tm_v, &tm_do);
+    if (warp == 12) bwd_mma<D, BF16>(p, sbase, tmem, ctl);
+    if (warp == 13 && lane == 0) bwd_load<D>(p, sbase, ctl, &tm_q, &tm_k, &tm_v, &tm_do);
     __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
