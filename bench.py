@@ -32,6 +32,8 @@ from tiled_online_softmax_03_b200.inputs import WORKLOADS, make_inputs  # noqa: 
 
 METRIC = ("attention fwd TFLOP/s (4·B·Hq·N²·d, ×½ causal) "
           "and % of B200 BF16 peak")
+METRIC_BWD = ("attention bwd TFLOP/s (2.5 × 4·B·Hq·N²·d, ×½ causal: five products per tile) "
+              "and % of B200 BF16 peak")
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0  # the same GEMM held under the 1 kW power cap
 KERNEL_SOURCES = ["tiled_online_softmax_03_b200/csrc/fa_fwd_sm100.cu",
@@ -299,6 +301,8 @@ def main():
                     help="B,Hq,Hk,N[,causal] replacing the workload's shape (other settings kept)")
     ap.add_argument("--bias", default="none", choices=["none", "heads", "full"],
                     help="additive bias [1, Hq, N, N] (heads) or [B, Hq, N, N] (full), fa_fwd_bias")
+    ap.add_argument("--backward", action="store_true",
+                    help="time fa_bwd (dQ, dK, dV for a seeded dO) instead of the forward")
     ap.add_argument("--splits", type=int, default=1,
                     help="K/V splits per Q tile pair (fa_fwd_splitkv; 1 = fa_fwd)")
     args = ap.parse_args()
@@ -357,8 +361,24 @@ def main():
         from tiled_online_softmax_03_b200.inputs import make_bias
         bias_t = make_bias(w, w.B if args.bias == "full" else 1, w.Hq, device=str(dev))
 
+    if args.backward and (bias_t is not None or args.splits > 1):
+        raise SystemExit("--backward takes neither --bias nor --splits")
+    bwd = None
+    if args.backward:
+        g = torch.Generator(device=str(dev)).manual_seed(w.seed + 4242)
+        dout = torch.randn(q.shape, generator=g, device=dev, dtype=torch.float32).to(q.dtype)
+        binding.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, key_pad_lens=lens, out=o, lse=lse)
+        bwd = {"dout": dout, "dq": torch.empty_like(q), "dk": torch.empty_like(k),
+               "dv": torch.empty_like(v),
+               "ws": torch.empty(binding.lib.fa_bwd_workspace_bytes(w.B, w.Hq, w.N, w.d),
+                                 dtype=torch.uint8, device=dev)}
+
     def call():
-        if bias_t is not None:
+        if bwd is not None:
+            binding.fa_bwd(q, k, v, o, lse, bwd["dout"], causal=w.causal, scale=w.scale,
+                           key_pad_lens=lens, dq=bwd["dq"], dk=bwd["dk"], dv=bwd["dv"],
+                           workspace=bwd["ws"], stream=stream.cuda_stream)
+        elif bias_t is not None:
             binding.fa_fwd_bias(q, k, v, bias_t, causal=w.causal, scale=w.scale, key_pad_lens=lens,
                                 out=o, lse=lse, stream=stream.cuda_stream)
         elif args.splits > 1:
@@ -412,6 +432,10 @@ def main():
     hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
     hlens = x["key_pad_lens"].pin_memory() if x["key_pad_lens"] is not None else None
     hbias = bias_t.cpu().pin_memory() if bias_t is not None else None
+    if bwd is not None:
+        hbo, hbl, hbd = (t.cpu().pin_memory() for t in (o, lse, bwd["dout"]))
+        hgrads = [torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                  for t in (bwd["dq"], bwd["dk"], bwd["dv"])]
     e2e_steps = max(1, min(args.e2e_steps, args.steps))
 
     def e2e_step():
@@ -422,6 +446,14 @@ def main():
             lens.copy_(hlens, non_blocking=True)
         if hbias is not None:
             bias_t.copy_(hbias, non_blocking=True)
+        if bwd is not None:
+            o.copy_(hbo, non_blocking=True)
+            lse.copy_(hbl, non_blocking=True)
+            bwd["dout"].copy_(hbd, non_blocking=True)
+            call()
+            for t, h in zip((bwd["dq"], bwd["dk"], bwd["dv"]), hgrads):
+                h.copy_(t, non_blocking=True)
+            return
         call()
         ho.copy_(o, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
@@ -441,13 +473,16 @@ def main():
         (hlens.numel() * 4 if hlens is not None else 0) + \
         (hbias.numel() * hbias.element_size() if hbias is not None else 0)
     d2h = ho.numel() * ho.element_size() + hl.numel() * 4
+    if bwd is not None:
+        h2d += sum(t.numel() * t.element_size() for t in (hbo, hbl, hbd))
+        d2h = sum(t.numel() * t.element_size() for t in hgrads)
 
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return
 
-    f = flops(w)
+    f = flops(w) * (2.5 if bwd is not None else 1.0)
     ms_per_step = total_ms / args.steps
     value = whole_job_tflops(f, world, ms_per_step)
     clk = clocks.summary()
@@ -459,7 +494,8 @@ def main():
     peak_src += ", sustained (sw_power_cap active in the timed region)" if peak == sustained and capped \
         else ", burst"
     achieved = f / (kern_avg * 1e-3) / 1e12
-    traffic = recorded_traffic(w.name) if args.splits == 1 and args.bias == "none" else None
+    traffic = recorded_traffic(w.name) if (args.splits == 1 and args.bias == "none"
+                                           and not args.backward) else None
     config = config_of(w, world)
     kernels = "fa_fwd_kernel"
     if args.splits > 1:
@@ -468,8 +504,11 @@ def main():
     if bias_t is not None:
         config["bias"] = list(bias_t.shape)
         kernels = "fa_fwd_kernel (bias)"
+    if bwd is not None:
+        config["pass"] = "backward"
+        kernels = "fa_bwd_pre_kernel + fa_bwd_kernel + fa_bwd_post_kernel"
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "metric": METRIC_BWD if bwd is not None else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
@@ -482,11 +521,11 @@ def main():
         "e2e": {"value": whole_job_tflops(f, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "steps": e2e_steps},
-        "gpu_launches": args.steps * (2 if args.splits > 1 else 1),
+        "gpu_launches": args.steps * (3 if bwd is not None else 2 if args.splits > 1 else 1),
         "clocks": clk,
         "device_status": status,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and bwd is None:
         line["cpu_baseline"] = {k2: v2 for k2, v2 in cpu_baseline(w).items()
                                 if k2 not in ("seconds", "heads")}
     print(json.dumps(line), flush=True)
