@@ -46,7 +46,7 @@ enum {
   BB_KV_EMPTY = 1,  // MMA -> TMA: the unit's MMAs no longer read K, V
   BB_QD_FULL = 2,   // [2] TMA -> MMA, softmax: Q, dO, LSE·log2e, D of a step
   BB_QD_EMPTY = 4,  // [2] MMA (commit) + 8 softmax warps -> TMA: stage read
-  BB_SDP_FULL = 6,  // MMA -> softmax: Sᵀ and dPᵀ in TMEM
+  BB_S_FULL = 6,    // MMA -> softmax: Sᵀ in TMEM
   BB_P_READY = 7,   // softmax -> MMA: Pᵀ, dSᵀ in TMEM and dSᵀ in smem
   BB_DQ_FULL = 8,   // MMA -> drain: dQ_part in TMEM
   BB_DQ_FREE = 9,   // drain -> MMA: dQ_part read
@@ -54,7 +54,8 @@ enum {
   BB_ACC_FREE = 11, // drain -> MMA: dK, dV read
   BB_DRAIN = 12,    // MMA drain on the abort path
   BB_STG_FREE = 13, // drain -> softmax: the dSᵀ tile, used as dQ staging, read by TMA
-  BB_COUNT = 14
+  BB_DP_FULL = 14,  // MMA -> softmax: dPᵀ in TMEM
+  BB_COUNT = 15
 };
 
 // Shared memory, no slack: the tiles need a 1 KB-aligned base, which the
@@ -220,12 +221,13 @@ __device__ void bwd_mma(const BParams& p, uint32_t sbase, uint32_t tmem, const C
       const uint32_t q_base = sbase + L::OFF_Q + stg * L::TILE;
       const uint32_t do_base = sbase + L::OFF_DO + stg * L::TILE;
       mma_kk(t_s, k_kmaj, sdesc(q_base, 16, 1024));                      // Sᵀ = K·Qᵀ
+      umma_commit_warp(bbar(sbase, BB_S_FULL));
       // dPᵀ overwrites the previous step's dQ_part: wait for the drain
       if (step_ct > 0 && !(ok = wait_bar_warp(bbar(sbase, BB_DQ_FREE), (step_ct - 1) & 1, c)))
         break;
       tc_fence_after();
       mma_kk(t_dp, v_kmaj, sdesc(do_base, 16, 1024));                    // dPᵀ = V·dOᵀ
-      umma_commit_warp(bbar(sbase, BB_SDP_FULL));
+      umma_commit_warp(bbar(sbase, BB_DP_FULL));
       if (!(ok = wait_bar_warp(bbar(sbase, BB_P_READY), step_ct & 1, c))) break;
       if (s == 0 && acc_units > 0 &&
           !(ok = wait_bar_warp(bbar(sbase, BB_ACC_FREE), (acc_units - 1) & 1, c)))
@@ -277,40 +279,54 @@ __device__ void bwd_softmax(const BParams& p, uint8_t* smem, uint32_t sbase, uin
     for (int s = 0; s < U.steps; ++s, ++step_ct) {
       const int stg = step_ct & 1, use = step_ct >> 1;
       if (!wait_bar_warp(bbar(sbase, BB_QD_FULL + stg), use & 1, c)) return;
-      if (!wait_bar_warp(bbar(sbase, BB_SDP_FULL), step_ct & 1, c)) return;
+      if (!wait_bar_warp(bbar(sbase, BB_S_FULL), step_ct & 1, c)) return;
       tc_fence_after();
       const int m = U.m_lo + s % U.nm;
       const float* lse2 = reinterpret_cast<const float*>(smem + L::OFF_LD + stg * 1024);
       const float* dsum = lse2 + 128;
       // queries j of the tile with key <= m·128 + j (causal), all if not causal
       const int q_first = p.causal ? key - m * BQ : 0;
-#pragma unroll 1
+      // phase 1 (while the tensor core computes dPᵀ): P for this thread's 64
+      // queries, kept in fp32 for dS, and written to TMEM as 16-bit pairs
+      float pf[64];
+#pragma unroll
       for (int cq = 0; cq < 2; ++cq) {
         const int cc = 2 * half + cq;  // 32-query chunk of the tile
-        uint32_t sv[32], dp[32];
+        uint32_t sv[32];
         tmem_ld_x32(t_s + 32 * cc, sv);
-        tmem_ld_x32(t_dp + 32 * cc, dp);
         tmem_wait_ld();
         reg_pin_x32(sv);
-        reg_pin_x32(dp);
-        uint32_t pk[16], dk2[16];
+        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float pv[2], dv[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int j = 32 * cc + 2 * i + h;
-            const bool allowed = key_ok && j >= q_first;
-            const float x = fmaf(__uint_as_float(sv[2 * i + h]), p.scale_log2, -lse2[j]);
-            pv[h] = allowed ? ex2_approx(x) : 0.f;
-            dv[h] = pv[h] * (__uint_as_float(dp[2 * i + h]) - dsum[j]);
-          }
-          pk[i] = round_pack<BF16>(pv[0], pv[1]);
-          dk2[i] = round_pack<BF16>(dv[0], dv[1]);
+        for (int i = 0; i < 32; ++i) {
+          const int j = 32 * cc + i;
+          const float x = fmaf(__uint_as_float(sv[i]), p.scale_log2, -lse2[j]);
+          pf[32 * cq + i] = (key_ok && j >= q_first) ? ex2_approx(x) : 0.f;
         }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = round_pack<BF16>(pf[32 * cq + 2 * i], pf[32 * cq + 2 * i + 1]);
         // packed pairs of half h go to columns 64·h + [0, 32): only columns this
         // thread has already read, never the other half's unread ones
         tmem_st_x16(t_s + 64 * half + 16 * cq, pk);
+      }
+      // phase 2: dS = P ⊙ (dP − D)
+      if (!wait_bar_warp(bbar(sbase, BB_DP_FULL), step_ct & 1, c)) return;
+      tc_fence_after();
+#pragma unroll
+      for (int cq = 0; cq < 2; ++cq) {
+        const int cc = 2 * half + cq;
+        uint32_t dp[32];
+        tmem_ld_x32(t_dp + 32 * cc, dp);
+        tmem_wait_ld();
+        reg_pin_x32(dp);
+        uint32_t dk2[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int j = 32 * cc + 2 * i;
+          const float d0 = pf[32 * cq + 2 * i] * (__uint_as_float(dp[2 * i]) - dsum[j]);
+          const float d1 = pf[32 * cq + 2 * i + 1] * (__uint_as_float(dp[2 * i + 1]) - dsum[j + 1]);
+          dk2[i] = round_pack<BF16>(d0, d1);
+        }
         tmem_st_x16(t_dp + 64 * half + 16 * cq, dk2);
       }
       tmem_wait_st();
@@ -356,22 +372,11 @@ __device__ void bwd_drain(const BParams& p, uint8_t* smem, uint32_t sbase, uint3
       // dQ_part through the 32 KB dSᵀ tile: two staging boxes of [128 rows][32
       // fp32]; each warp stages its own 32 rows and its lane 0 adds that 4 KB
       // slab into dQ by TMA (no cross-warp barrier). Row r, 16-byte chunk i
-      // sits at chunk i ^ (r & 7) of its 128-byte row (128-byte swizzle).
-#pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t v[32];
-        tmem_ld_x32(t_row + 128 + 32 * cc, v);
-        tmem_wait_ld();
-        reg_pin_x32(v);
-        if (cc == D / 32 - 1) {
-          tc_fence_before();
-          mbar_arrive(bbar(sbase, BB_DQ_FREE));
-        }
-        if (cc >= 2) {  // this box was staged two chunks ago: has TMA read it?
-          if (lane == 0) bulk_wait_group_read<1>();
-          __syncwarp();
-        }
-        const uint32_t slab = L::OFF_DS + (cc & 1) * STG_BOX + wl * 32 * 128;
+      // sits at chunk i ^ (r & 7) of its 128-byte row (128-byte swizzle). All
+      // TMEM reads come before any wait on TMA, so the MMA warp gets the
+      // columns back (DQ_FREE) as early as possible.
+      auto stage = [&](const uint32_t* v, int box, int cc) {
+        const uint32_t slab = L::OFF_DS + box * STG_BOX + wl * 32 * 128;
         uint8_t* row = smem + slab + (r & 31) * 128;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
@@ -379,10 +384,27 @@ __device__ void bwd_drain(const BParams& p, uint8_t* smem, uint32_t sbase, uint3
               make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-          tma_reduce_add_3d(tm_dq, sbase + slab, 32 * cc, m * BQ + wl * 32, head);
-          bulk_commit_group();
+        if (lane == 0) tma_reduce_add_3d(tm_dq, sbase + slab, 32 * cc, m * BQ + wl * 32, head);
+      };
+#pragma unroll 1
+      for (int pair = 0; pair < D / 64; ++pair) {
+        uint32_t a[32], b[32];
+        tmem_ld_x32(t_row + 128 + 64 * pair, a);
+        tmem_ld_x32(t_row + 128 + 64 * pair + 32, b);
+        tmem_wait_ld();
+        reg_pin_x32(a);
+        reg_pin_x32(b);
+        if (pair == D / 64 - 1) {
+          tc_fence_before();
+          mbar_arrive(bbar(sbase, BB_DQ_FREE));
         }
+        if (pair > 0) {  // the previous pair's staging read by TMA?
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+        }
+        stage(a, 0, 2 * pair);
+        stage(b, 1, 2 * pair + 1);
+        if (lane == 0) bulk_commit_group();
       }
       if (lane == 0) {
         bulk_wait_group_read<0>();
@@ -460,7 +482,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bbar(sbase, BB_QD_FULL + s), 1);
       mbar_init(bbar(sbase, BB_QD_EMPTY + s), 1 + 8);  // MMA commit + one per softmax warp
     }
-    mbar_init(bbar(sbase, BB_SDP_FULL), 1);
+    mbar_init(bbar(sbase, BB_S_FULL), 1);
+    mbar_init(bbar(sbase, BB_DP_FULL), 1);
     mbar_init(bbar(sbase, BB_P_READY), 256);
     mbar_init(bbar(sbase, BB_DQ_FULL), 1);
     mbar_init(bbar(sbase, BB_DQ_FREE), 128);
@@ -487,11 +510,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Ctl ctl{abort_flag, p.timeout_ns};
+  // Register split: 2×152 (softmax) + 104 (drain) + 104 (MMA, loads) = 4 × 128.
   if (warp < 8) {
+    setmaxnreg_inc<152>();
     bwd_softmax<D, BF16>(p, bsmem, sbase, tmem, ctl);
   } else if (warp < 12) {
+    setmaxnreg_dec<104>();
     bwd_drain<D, BF16>(p, bsmem, sbase, tmem, ctl, &tm_dq);
   } else {
+    setmaxnreg_dec<104>();
     if (warp == 12) bwd_mma<D, BF16>(p, sbase, tmem, ctl);
     if (warp == 13 && lane == 0) bwd_load<D>(p, sbase, ctl, &tm_q, &tm_k, &tm_v, &tm_do);
     __syncwarp();

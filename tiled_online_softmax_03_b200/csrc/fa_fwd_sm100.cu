@@ -1530,6 +1530,14 @@ int bwd_launch(const void* q, const void* k, const void* v, const void* o, const
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES) !=
           cudaSuccess)
         return fail(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
+      cudaFuncAttributes fa_attr;
+      if (cudaFuncGetAttributes(&fa_attr, kern) != cudaSuccess)
+        return fail(FA_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(cudaGetLastError()));
+      // The setmaxnreg split (2×152 + 104 + 104 per 128 threads) needs exactly
+      // 128 registers per thread at launch.
+      if (fa_attr.numRegs != 128)
+        return fail(FA_ERR_UNSUPPORTED, "backward kernel built with %d registers per thread, need 128",
+                    fa_attr.numRegs);
       info.bwd_attr_set[slot] = true;
     }
   }
