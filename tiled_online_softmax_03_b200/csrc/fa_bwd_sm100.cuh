@@ -289,6 +289,8 @@ __device__ void bwd_softmax(const BParams& p, uint8_t* smem, uint32_t sbase, uin
       // phase 1 (while the tensor core computes dPᵀ): P for this thread's 64
       // queries, kept in fp32 for dS, and written to TMEM as 16-bit pairs
       float pf[64];
+      // every query of this thread's half allowed (off the causal diagonal)?
+      const bool all_ok = key_ok && q_first <= 64 * half;
 #pragma unroll
       for (int cq = 0; cq < 2; ++cq) {
         const int cc = 2 * half + cq;  // 32-query chunk of the tile
@@ -297,11 +299,29 @@ __device__ void bwd_softmax(const BParams& p, uint8_t* smem, uint32_t sbase, uin
         tmem_wait_ld();
         reg_pin_x32(sv);
         uint32_t pk[16];
+        const float4* l4 = reinterpret_cast<const float4*>(lse2 + 32 * cc);
+        if (all_ok) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int j = 32 * cc + i;
-          const float x = fmaf(__uint_as_float(sv[i]), p.scale_log2, -lse2[j]);
-          pf[32 * cq + i] = (key_ok && j >= q_first) ? ex2_approx(x) : 0.f;
+          for (int g = 0; g < 8; ++g) {
+            const float4 l = l4[g];
+            const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              pf[32 * cq + 4 * g + e] =
+                  ex2_approx(fmaf(__uint_as_float(sv[4 * g + e]), p.scale_log2, -lv[e]));
+          }
+        } else {
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const float4 l = l4[g];
+            const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = 32 * cc + 4 * g + e;
+              const float x = fmaf(__uint_as_float(sv[4 * g + e]), p.scale_log2, -lv[e]);
+              pf[32 * cq + 4 * g + e] = (key_ok && j >= q_first) ? ex2_approx(x) : 0.f;
+            }
+          }
         }
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[i] = round_pack<BF16>(pf[32 * cq + 2 * i], pf[32 * cq + 2 * i + 1]);
@@ -320,12 +340,15 @@ __device__ void bwd_softmax(const BParams& p, uint8_t* smem, uint32_t sbase, uin
         tmem_wait_ld();
         reg_pin_x32(dp);
         uint32_t dk2[16];
+        const float4* d4 = reinterpret_cast<const float4*>(dsum + 32 * cc);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int j = 32 * cc + 2 * i;
-          const float d0 = pf[32 * cq + 2 * i] * (__uint_as_float(dp[2 * i]) - dsum[j]);
-          const float d1 = pf[32 * cq + 2 * i + 1] * (__uint_as_float(dp[2 * i + 1]) - dsum[j + 1]);
-          dk2[i] = round_pack<BF16>(d0, d1);
+        for (int g = 0; g < 8; ++g) {
+          const float4 dd = d4[g];
+          const int i = 4 * g;
+          dk2[2 * g] = round_pack<BF16>(pf[32 * cq + i] * (__uint_as_float(dp[i]) - dd.x),
+                                        pf[32 * cq + i + 1] * (__uint_as_float(dp[i + 1]) - dd.y));
+          dk2[2 * g + 1] = round_pack<BF16>(pf[32 * cq + i + 2] * (__uint_as_float(dp[i + 2]) - dd.z),
+                                            pf[32 * cq + i + 3] * (__uint_as_float(dp[i + 3]) - dd.w));
         }
         tmem_st_x16(t_dp + 64 * half + 16 * cq, dk2);
       }
@@ -386,24 +409,22 @@ __device__ void bwd_drain(const BParams& p, uint8_t* smem, uint32_t sbase, uint3
         __syncwarp();
         if (lane == 0) tma_reduce_add_3d(tm_dq, sbase + slab, 32 * cc, m * BQ + wl * 32, head);
       };
-#pragma unroll 1
+      uint32_t v[D / 32][32];
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) tmem_ld_x32(t_row + 128 + 32 * cc, v[cc]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) reg_pin_x32(v[cc]);
+      tc_fence_before();
+      mbar_arrive(bbar(sbase, BB_DQ_FREE));
+#pragma unroll
       for (int pair = 0; pair < D / 64; ++pair) {
-        uint32_t a[32], b[32];
-        tmem_ld_x32(t_row + 128 + 64 * pair, a);
-        tmem_ld_x32(t_row + 128 + 64 * pair + 32, b);
-        tmem_wait_ld();
-        reg_pin_x32(a);
-        reg_pin_x32(b);
-        if (pair == D / 64 - 1) {
-          tc_fence_before();
-          mbar_arrive(bbar(sbase, BB_DQ_FREE));
-        }
         if (pair > 0) {  // the previous pair's staging read by TMA?
           if (lane == 0) bulk_wait_group_read<0>();
           __syncwarp();
         }
-        stage(a, 0, 2 * pair);
-        stage(b, 1, 2 * pair + 1);
+        stage(v[2 * pair], 0, 2 * pair);
+        stage(v[2 * pair + 1], 1, 2 * pair + 1);
         if (lane == 0) bulk_commit_group();
       }
       if (lane == 0) {
@@ -510,15 +531,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Ctl ctl{abort_flag, p.timeout_ns};
-  // Register split: 2×152 (softmax) + 104 (drain) + 104 (MMA, loads) = 4 × 128.
+  // Register split: 2×136 (softmax) + 144 (drain: a whole dQ_part row in
+  // registers) + 96 (MMA, loads) = 4 × 128.
   if (warp < 8) {
-    setmaxnreg_inc<152>();
+    setmaxnreg_inc<136>();
     bwd_softmax<D, BF16>(p, bsmem, sbase, tmem, ctl);
   } else if (warp < 12) {
-    setmaxnreg_dec<104>();
+    setmaxnreg_inc<144>();
     bwd_drain<D, BF16>(p, bsmem, sbase, tmem, ctl, &tm_dq);
   } else {
-    setmaxnreg_dec<104>();
+    setmaxnreg_dec<96>();
     if (warp == 12) bwd_mma<D, BF16>(p, sbase, tmem, ctl);
     if (warp == 13 && lane == 0) bwd_load<D>(p, sbase, ctl, &tm_q, &tm_k, &tm_v, &tm_do);
     __syncwarp();

@@ -1533,7 +1533,7 @@ int bwd_launch(const void* q, const void* k, const void* v, const void* o, const
       cudaFuncAttributes fa_attr;
       if (cudaFuncGetAttributes(&fa_attr, kern) != cudaSuccess)
         return fail(FA_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(cudaGetLastError()));
-      // The setmaxnreg split (2×152 + 104 + 104 per 128 threads) needs exactly
+      // The setmaxnreg split (2×136 + 144 + 96 per 128 threads) needs exactly
       // 128 registers per thread at launch.
       if (fa_attr.numRegs != 128)
         return fail(FA_ERR_UNSUPPORTED, "backward kernel built with %d registers per thread, need 128",
