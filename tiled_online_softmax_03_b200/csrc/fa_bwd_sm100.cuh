@@ -13,7 +13,7 @@
 // dV accumulate in tensor memory over every (query head of the group, query
 // tile m) that sees the block — one "step" each — and are written once at the
 // unit's end, so they need no atomics. dQ of a step is a partial sum over this
-// key block only; it is added into an fp32 buffer with vector reductions and
+// key block only; it is added into an fp32 buffer by TMA reduce-add and
 // scaled and rounded by a final kernel.
 //
 // Per step (Q, dO, LSE·log2e and D of query tile m staged by TMA, two stages):

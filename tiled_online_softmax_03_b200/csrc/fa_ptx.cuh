@@ -86,13 +86,6 @@ __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint
       ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
-// Four fp32 atomic adds to global memory at a 16-byte aligned address (no
-// return value; sm_90 and later).
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
 // 3-D tiled reduce-add shared -> global (f32 add into the tensor; rows past
 // the extent are clipped).
 __device__ __forceinline__ void tma_reduce_add_3d(const void* map, uint32_t src, int c0, int c1,
@@ -101,10 +94,6 @@ __device__ __forceinline__ void tma_reduce_add_3d(const void* map, uint32_t src,
       "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
       ::"l"(map), "r"(src), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
-}
-// Barrier over the `count` threads of a warp group that use named barrier `id`.
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
