@@ -301,6 +301,8 @@ def main():
                     help="B,Hq,Hk,N[,causal] replacing the workload's shape (other settings kept)")
     ap.add_argument("--bias", default="none", choices=["none", "heads", "full"],
                     help="additive bias [1, Hq, N, N] (heads) or [B, Hq, N, N] (full), fa_fwd_bias")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time fa_fwd_fp8 on the workload's inputs quantised per tensor to E4M3")
     ap.add_argument("--backward", action="store_true",
                     help="time fa_bwd (dQ, dK, dV for a seeded dO) instead of the forward")
     ap.add_argument("--splits", type=int, default=1,
@@ -363,6 +365,18 @@ def main():
 
     if args.backward and (bias_t is not None or args.splits > 1):
         raise SystemExit("--backward takes neither --bias nor --splits")
+    f8 = None
+    if args.fp8:
+        if args.backward or bias_t is not None or args.splits > 1:
+            raise SystemExit("--fp8 is a forward of its own: no --backward, --bias or --splits")
+        f8 = {}
+        for n, t in (("q", q), ("k", k), ("v", v)):
+            amax = float(t.float().abs().max())
+            f8[n + "s"] = amax / 448.0 if amax > 0 else 1.0
+            f8[n] = (t.float() / f8[n + "s"]).to(torch.float8_e4m3fn)
+        f8["o"] = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+        f8["ws"] = torch.empty(binding.lib.fa_fwd_fp8_workspace_bytes(w.B, w.Hk, w.N, w.d),
+                               dtype=torch.uint8, device=dev)
     bwd = None
     if args.backward:
         g = torch.Generator(device=str(dev)).manual_seed(w.seed + 4242)
@@ -374,7 +388,11 @@ def main():
                                  dtype=torch.uint8, device=dev)}
 
     def call():
-        if bwd is not None:
+        if f8 is not None:
+            binding.fa_fwd_fp8(f8["q"], f8["k"], f8["v"], f8["qs"], f8["ks"], f8["vs"],
+                               causal=w.causal, scale=w.scale, key_pad_lens=lens, out=f8["o"],
+                               lse=lse, workspace=f8["ws"], stream=stream.cuda_stream)
+        elif bwd is not None:
             binding.fa_bwd(q, k, v, o, lse, bwd["dout"], causal=w.causal, scale=w.scale,
                            key_pad_lens=lens, dq=bwd["dq"], dk=bwd["dk"], dv=bwd["dv"],
                            workspace=bwd["ws"], stream=stream.cuda_stream)
@@ -432,6 +450,9 @@ def main():
     hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
     hlens = x["key_pad_lens"].pin_memory() if x["key_pad_lens"] is not None else None
     hbias = bias_t.cpu().pin_memory() if bias_t is not None else None
+    if f8 is not None:
+        hf8 = {n: f8[n].cpu().pin_memory() for n in ("q", "k", "v")}
+        ho8 = torch.empty(f8["o"].shape, dtype=torch.bfloat16).pin_memory()
     if bwd is not None:
         hbo, hbl, hbd = (t.cpu().pin_memory() for t in (o, lse, bwd["dout"]))
         hgrads = [torch.empty(t.shape, dtype=t.dtype).pin_memory()
@@ -446,6 +467,13 @@ def main():
             lens.copy_(hlens, non_blocking=True)
         if hbias is not None:
             bias_t.copy_(hbias, non_blocking=True)
+        if f8 is not None:
+            for n in ("q", "k", "v"):
+                f8[n].copy_(hf8[n], non_blocking=True)
+            call()
+            ho8.copy_(f8["o"], non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+            return
         if bwd is not None:
             o.copy_(hbo, non_blocking=True)
             lse.copy_(hbl, non_blocking=True)
@@ -476,6 +504,9 @@ def main():
     if bwd is not None:
         h2d += sum(t.numel() * t.element_size() for t in (hbo, hbl, hbd))
         d2h = sum(t.numel() * t.element_size() for t in hgrads)
+    if f8 is not None:
+        h2d = sum(t.numel() * t.element_size() for t in hf8.values()) + \
+            (hlens.numel() * 4 if hlens is not None else 0)
 
     if world > 1:
         dist.destroy_process_group()
@@ -490,12 +521,15 @@ def main():
     # Burst peak for a kernel timed before the power cap engages; the sustained
     # one once the timed region ran under sw_power_cap (a long back-to-back loop).
     capped = "sw_power_cap" in clk.get("reasons", [])
+    if f8 is not None:  # E4M3 dense rate: the measured bf16 peaks × 2 (nominal 4.5 / 2.25 PFLOP/s)
+        burst, sustained = 2 * burst, (2 * sustained if sustained else None)
+        peak_src += " × 2 for E4M3 (nominal fp8/bf16 ratio)"
     peak = sustained if (capped and sustained) else burst
     peak_src += ", sustained (sw_power_cap active in the timed region)" if peak == sustained and capped \
         else ", burst"
     achieved = f / (kern_avg * 1e-3) / 1e12
     traffic = recorded_traffic(w.name) if (args.splits == 1 and args.bias == "none"
-                                           and not args.backward) else None
+                                           and not args.backward and not args.fp8) else None
     config = config_of(w, world)
     kernels = "fa_fwd_kernel"
     if args.splits > 1:
@@ -504,6 +538,9 @@ def main():
     if bias_t is not None:
         config["bias"] = list(bias_t.shape)
         kernels = "fa_fwd_kernel (bias)"
+    if f8 is not None:
+        config["in_dtype"] = "e4m3 (per-tensor descale), O bf16"
+        kernels = "fa_transpose_u8_kernel + fa_fwd_kernel (FP8)"
     if bwd is not None:
         config["pass"] = "backward"
         kernels = "fa_bwd_pre_kernel + fa_bwd_kernel + fa_bwd_post_kernel"
@@ -511,7 +548,7 @@ def main():
         "metric": METRIC_BWD if bwd is not None else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": w.dtype, "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
+        "dtype": "e4m3" if f8 is not None else w.dtype, "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
         "config": config,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
@@ -521,11 +558,12 @@ def main():
         "e2e": {"value": whole_job_tflops(f, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "steps": e2e_steps},
-        "gpu_launches": args.steps * (3 if bwd is not None else 2 if args.splits > 1 else 1),
+        "gpu_launches": args.steps * (3 if bwd is not None else 2 if (args.splits > 1 or f8 is not None)
+                                      else 1),
         "clocks": clk,
         "device_status": status,
     }
-    if world == 1 and not args.no_cpu_baseline and bwd is None:
+    if world == 1 and not args.no_cpu_baseline and bwd is None and f8 is None:
         line["cpu_baseline"] = {k2: v2 for k2, v2 in cpu_baseline(w).items()
                                 if k2 not in ("seconds", "heads")}
     print(json.dumps(line), flush=True)

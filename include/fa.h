@@ -173,6 +173,36 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
 /* Workspace bytes fa_bwd needs (0 for invalid arguments). */
 size_t fa_bwd_workspace_bytes(int B, int Hq, int N, int d);
 
+/*
+ * fa_fwd_fp8 — fa_fwd on E4M3 (8-bit float) inputs with per-tensor descale
+ * factors: the decoded inputs are Q = q·q_descale, K = k·k_descale,
+ * V = v·v_descale, and O = softmax(scale·QKᵀ + mask)·V is written as bfloat16
+ * with LSE in fp32 as fa_fwd. (The GQA page "深度探索Flash-Attention中GQA性能
+ * 调优技术解析", section "混合精度训练的内存优化", names FP8 for halving the
+ * memory traffic; "FlashAttention (VI)" attributes FP8 to FlashAttention-3.)
+ * Q·Kᵀ and P·V run on the tensor core in E4M3 with fp32 accumulation; P is
+ * rounded to E4M3 for P·V and the row sums use the same rounded values.
+ *
+ *   q, k, v          device pointers to E4M3 bytes, layouts [B,H,N,d] as fa_fwd.
+ *   q_descale, k_descale, v_descale  finite factors > 0.
+ *   o                [B, Hq, N, d] bfloat16, written; lse as fa_fwd.
+ *   d                128 only; N a multiple of 16 (V is transposed into the
+ *                    workspace and loaded by TMA with N-byte rows); other values
+ *                    return FA_ERR_UNSUPPORTED.
+ *   workspace        device pointer, 256-byte aligned, at least
+ *                    fa_fwd_fp8_workspace_bytes(B, Hk, N, d) bytes (the
+ *                    transposed V); scratch after the call; one per call in flight.
+ *   other arguments  as for fa_fwd.
+ * Enqueues two kernels on `stream`. Returns FA_OK or a negative fa_status.
+ */
+int fa_fwd_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,
+               float v_descale, void* o, float* lse, int B, int Hq, int Hk, int N, int d,
+               float scale, int causal, const int32_t* key_pad_lens, void* workspace,
+               size_t workspace_bytes, void* stream);
+
+/* Workspace bytes fa_fwd_fp8 needs (0 for unsupported arguments). */
+size_t fa_fwd_fp8_workspace_bytes(int B, int Hk, int N, int d);
+
 /* Workspace bytes fa_fwd_splitkv needs: B·Hq·N·num_splits·(d + 1) floats,
  * each part rounded up to 256 bytes; 0 for num_splits == 1 and for invalid
  * arguments. */

@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["FaError", "fa_fwd", "fa_bwd", "fa_fwd_bias", "fa_fwd_splitkv", "splitkv_workspace_bytes", "load_library", "lib", "FA_OK", "FA_ERR_INVALID_ARG",
+__all__ = ["FaError", "fa_fwd", "fa_bwd", "fa_fwd_fp8", "fa_fwd_bias", "fa_fwd_splitkv", "splitkv_workspace_bytes", "load_library", "lib", "FA_OK", "FA_ERR_INVALID_ARG",
            "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT"]
 
 FA_OK = 0
@@ -48,6 +48,11 @@ def load_library(path=LIB_PATH):
     L.fa_bwd.restype = c_int
     L.fa_bwd_workspace_bytes.argtypes = [c_int] * 4
     L.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
+    L.fa_fwd_fp8.argtypes = [c_void_p] * 3 + [c_float] * 3 + [c_void_p, c_void_p] + [c_int] * 5 + \
+        [c_float, c_int, c_void_p, c_void_p, ctypes.c_size_t, c_void_p]
+    L.fa_fwd_fp8.restype = c_int
+    L.fa_fwd_fp8_workspace_bytes.argtypes = [c_int] * 4
+    L.fa_fwd_fp8_workspace_bytes.restype = ctypes.c_size_t
     L.fa_fwd_bias.argtypes = [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p,
                               c_void_p, c_int, c_int, c_int, c_int, c_int, c_float, c_int,
                               c_void_p, c_void_p, c_int]
@@ -195,6 +200,47 @@ def fa_bwd(q, k, v, o, lse, dout, causal=False, scale=None, key_pad_lens=None, d
                          workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                          stream, _DTYPES[q.dtype]))
     return dq, dk, dv
+
+
+def fa_fwd_fp8(q, k, v, q_descale, k_descale, v_descale, causal=False, scale=None,
+               key_pad_lens=None, out=None, lse=None, return_lse=True, workspace=None, stream=None):
+    """Attention forward on E4M3 inputs (torch.float8_e4m3fn, values = stored × descale).
+
+    O is bfloat16. ``scale`` defaults to 1/sqrt(d) and multiplies the decoded
+    scores. The workspace (a transposed copy of V) is allocated when None.
+    """
+    fp8 = getattr(torch, "float8_e4m3fn", None)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4 or t.dtype != fp8:
+            raise FaError(FA_ERR_INVALID_ARG,
+                          f"{name} must be a contiguous 4-D CUDA tensor of torch.float8_e4m3fn")
+    B, Hq, N, d = q.shape
+    Hk = k.shape[1]
+    if tuple(k.shape) != (B, Hk, N, d) or tuple(v.shape) != (B, Hk, N, d):
+        raise FaError(FA_ERR_INVALID_ARG, "k and v must be [B, Hk, N, d] matching q")
+    if out is None:
+        out = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    if key_pad_lens is not None and (key_pad_lens.dtype != torch.int32 or not key_pad_lens.is_cuda
+                                     or key_pad_lens.numel() != B):
+        raise FaError(FA_ERR_INVALID_ARG, "key_pad_lens must be an int32 CUDA tensor [B]")
+    if scale is None:
+        scale = float(d) ** -0.5
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    need = lib.fa_fwd_fp8_workspace_bytes(B, Hk, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        check(lib.fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), float(q_descale),
+                             float(k_descale), float(v_descale), out.data_ptr(),
+                             lse.data_ptr() if lse is not None else None, B, Hq, Hk, N, d,
+                             float(scale), 1 if causal else 0,
+                             key_pad_lens.data_ptr() if key_pad_lens is not None else None,
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                             stream))
+    return (out, lse) if return_lse else out
 
 
 def splitkv_workspace_bytes(B, Hq, N, d, num_splits):

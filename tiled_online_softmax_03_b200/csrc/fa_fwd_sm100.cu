@@ -81,11 +81,14 @@ enum {
 // Shared memory: barriers and flags first, then 1 KB-aligned tiles. With an
 // additive bias the K/V ring is halved to make room for one 128×128 16-bit
 // bias tile per Q tile.
-template <int D, bool BIAS = false>
+// MODE: 0 = plain, 1 = additive bias, 2 = FP8 (E4M3 Q, K, V).
+template <int D, int MODE = 0>
 struct Layout {
-  static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int STAGES = BIAS ? ((D == 128) ? 2 : 4) : ((D == 128) ? 4 : 8);
+  static constexpr bool BIAS = MODE == 1, FP8 = MODE == 2;
+  static constexpr int ELEM = FP8 ? 1 : 2;  // bytes per Q, K, V element
+  static constexpr int Q_BYTES = BM * D * ELEM;
+  static constexpr int KV_BYTES = BN * D * ELEM;
+  static constexpr int STAGES = BIAS ? ((D == 128) ? 2 : 4) : ((D == 128 && !FP8) ? 4 : 8);
   static constexpr int BIAS_BYTES = BIAS ? BM * BN * 2 : 0;
   static constexpr int NUM_BARS = BAR_KV + 2 * STAGES;
   static constexpr int OFF_BAR = 0;
@@ -109,6 +112,7 @@ struct Params {
   float* lse;
   float* o_part;    // split-KV: [splits][B·Hq][N][d] fp32 partial O (normalised), else null
   float* lse_part;  // split-KV: [splits][B·Hq][N] fp32 partial LSE
+  float o_scale;    // FP8 mode: the V descale, applied to O in the epilogue
   int bias_bmul;    // bias mode: bias plane of (b, hq) is (b·bias_bmul)·bias_H + hq·bias_hmul
   int bias_hmul;
   int bias_H;
@@ -180,10 +184,13 @@ __device__ __forceinline__ bool next_unit(const Params& p, int it, Unit& U) {
 }
 
 // ============================================================ TMA producer
-template <int D, bool BIAS>
+template <int D, int MODE>
 __device__ void role_load(const Params& p, uint32_t sbase, const Ctl& c, const CUtensorMap* tm_q,
                           const CUtensorMap* tm_k, const CUtensorMap* tm_v) {
-  using L = Layout<D, BIAS>;
+  using L = Layout<D, MODE>;
+  constexpr bool BIAS = L::BIAS, FP8 = L::FP8;
+  (void)BIAS;
+  (void)FP8;
   uint32_t qe_ph[2] = {0, 0};
   int st = 0;
   uint32_t kv_ph = 0;
@@ -201,8 +208,10 @@ __device__ void role_load(const Params& p, uint32_t sbase, const Ctl& c, const C
       last_q_ph[t] = (armed_q >> t & 1) ? last_q_ph[t] ^ 1 : 0;
       armed_q |= 1u << t;
       const int head = U.b * p.s.Hq + U.hq[t];
-      for (int bx = 0; bx < D / 64; ++bx)
-        tma_load_3d(sbase + L::OFF_Q + t * L::Q_BYTES + bx * SW128_BOX_BYTES, tm_q, bx * 64,
+      // a 128-byte-wide box: 64 16-bit or 128 8-bit columns
+      constexpr int BOX_COLS = 128 / L::ELEM;
+      for (int bx = 0; bx < D / BOX_COLS; ++bx)
+        tma_load_3d(sbase + L::OFF_Q + t * L::Q_BYTES + bx * SW128_BOX_BYTES, tm_q, bx * BOX_COLS,
                     U.mb[t] * BM, head, full);
     }
     const int kv_head = U.b * p.s.Hk + U.hk;
@@ -213,10 +222,19 @@ __device__ void role_load(const Params& p, uint32_t sbase, const Ctl& c, const C
         mbar_arrive_expect_tx(full, L::KV_BYTES);
         last_kv_ph[st] = kv_ph;
         armed_kv |= 1u << st;
-        const CUtensorMap* map = which ? tm_v : tm_k;
-        for (int bx = 0; bx < D / 64; ++bx)
-          tma_load_3d(sbase + L::OFF_KV + st * L::KV_BYTES + bx * SW128_BOX_BYTES, map, bx * 64,
-                      j * BN, kv_head, full);
+        if constexpr (FP8) {
+          // K_j: [128 keys][128 8-bit d] one box. V_j from the transposed copy
+          // Vᵀ [d][N]: d rows × keys j·128 .. +127 (K-major for the P·V product).
+          if (which)
+            tma_load_3d(sbase + L::OFF_KV + st * L::KV_BYTES, tm_v, j * BN, 0, kv_head, full);
+          else
+            tma_load_3d(sbase + L::OFF_KV + st * L::KV_BYTES, tm_k, 0, j * BN, kv_head, full);
+        } else {
+          const CUtensorMap* map = which ? tm_v : tm_k;
+          for (int bx = 0; bx < D / 64; ++bx)
+            tma_load_3d(sbase + L::OFF_KV + st * L::KV_BYTES + bx * SW128_BOX_BYTES, map, bx * 64,
+                        j * BN, kv_head, full);
+        }
         if (++st == L::STAGES) {
           st = 0;
           kv_ph ^= 1;
@@ -274,11 +292,16 @@ __device__ void role_bias_load(const Params& p, uint32_t sbase, const Ctl& c,
 
 // Run by the whole of warp 12, converged; one elected lane issues each
 // tcgen05 instruction.
-template <int D, bool BF16, bool BIAS>
+template <int D, bool BF16, int MODE>
 __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const Ctl& c) {
-  using L = Layout<D, BIAS>;
-  constexpr uint32_t IDESC_QK = idesc_f16(BF16, BN, false);  // S = Q·Kᵀ, both K-major
-  constexpr uint32_t IDESC_PV = idesc_f16(BF16, D, true);    // O += P·V, V is MN-major
+  using L = Layout<D, MODE>;
+  constexpr bool BIAS = L::BIAS, FP8 = L::FP8;
+  (void)BIAS;
+  (void)FP8;
+  // S = Q·Kᵀ, both K-major; O += P·V with V MN-major (16-bit) or, for FP8, Vᵀ
+  // K-major (E4M3 is format 0 of kind::f8f6f4, as fp16 is of kind::f16)
+  constexpr uint32_t IDESC_QK = idesc_f16(BF16 && !FP8, BN, false);
+  constexpr uint32_t IDESC_PV = idesc_f16(BF16 && !FP8, D, !FP8);
   int st = 0;
   uint32_t kv_ph = 0;
   bool ok = true;
@@ -291,11 +314,18 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
   // the accumulate flag is a compile-time constant except on the first step.
   const uint64_t q_desc0 = sdesc(sbase + L::OFF_Q, 16, 1024);
   const uint64_t kv_desc0 = sdesc(sbase + L::OFF_KV, 16, 1024);
-  const uint64_t v_desc0 = sdesc(sbase + L::OFF_KV, SW128_BOX_BYTES, 1024);
+  const uint64_t v_desc0 = FP8 ? sdesc(sbase + L::OFF_KV, 16, 1024)
+                                : sdesc(sbase + L::OFF_KV, SW128_BOX_BYTES, 1024);
   auto issue_qk = [&](int t, int kst) {
     const uint64_t qd = q_desc0 + (uint64_t)((t * L::Q_BYTES) >> 4);
     const uint64_t kd = kv_desc0 + (uint64_t)((kst * L::KV_BYTES) >> 4);
     const uint32_t d_s = tmem + S_COL[t];
+    if constexpr (FP8) {  // K = 32 bytes per MMA, all inside one 128-byte row
+      umma_ss_f8_warp(d_s, qd, kd, IDESC_QK, 0u);
+#pragma unroll
+      for (int k = 1; k < D / 32; ++k) umma_ss_f8_warp(d_s, qd + 2 * k, kd + 2 * k, IDESC_QK, 1u);
+      return;
+    }
     umma_ss_warp(d_s, qd, kd, IDESC_QK, 0u);
 #pragma unroll
     for (int k = 1; k < D / 16; ++k) {
@@ -310,6 +340,14 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
     const uint64_t vd = v_desc0 + (uint64_t)((vst * L::KV_BYTES) >> 4);
     const uint32_t d_o = tmem + TmemO<D>::col(t);
     const uint32_t a_p = tmem + S_COL[t];
+    if constexpr (FP8) {
+      // P: 32 keys = 8 TMEM columns (four E4M3 values per column); Vᵀ rows
+      // hold keys, 32 keys = 32 bytes of each 128-byte row
+#pragma unroll
+      for (int k = 2 * h; k < 2 * h + 2; ++k)
+        umma_ts_f8_warp(d_o, a_p + k * 8, vd + 2 * k, IDESC_PV, k == 0 ? acc : 1u);
+      return;
+    }
     const int k0 = h * (BN / 32);
     umma_ts_warp(d_o, a_p + k0 * 8, vd + ((k0 * 16 * 128) >> 4), IDESC_PV, acc);
 #pragma unroll
@@ -553,6 +591,45 @@ __device__ __forceinline__ float exp_store(const uint32_t (&s)[BN], float sl2, f
   return f2_lo(e2) + f2_hi(e2);
 }
 
+// FP8 form of exp_store: P rounded to E4M3 (four keys per TMEM column, 32
+// columns per tile), first 64 keys stored and signalled early. Returns the sum
+// of the unrounded P (LSE) and, in *qsum, the sum of the rounded P — the exact
+// denominator of the P·V product the tensor core forms from them.
+template <bool MASKED>
+__device__ __forceinline__ float exp_store_f8(const uint32_t (&s)[BN], float sl2, float mref,
+                                              uint32_t t_p, uint32_t half_bar, float* qsum) {
+  const uint64_t k2 = f2_pack(sl2, sl2), nm2 = f2_pack(-mref, -mref);
+  uint64_t acc[2] = {0, 0}, accq[2] = {0, 0};
+  uint32_t pk[BN / 4];
+#pragma unroll
+  for (int w = 0; w < BN / 4; ++w) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = 2 * w + h;
+      const uint64_t x = ((uint64_t)s[2 * i + 1] << 32) | s[2 * i];
+      const uint64_t y = MASKED ? fadd2(x, nm2) : ffma2(x, k2, nm2);
+      const float p0 = ex2_approx(f2_lo(y)), p1 = ex2_approx(f2_hi(y));
+      acc[h] = fadd2(acc[h], f2_pack(p0, p1));
+      const uint32_t q = e4m3x2(p0, p1);
+      accq[h] = fadd2(accq[h], e4m3x2_to_f2(q));
+      word |= q << (16 * h);
+    }
+    pk[w] = word;
+    if (w == BN / 8 - 1) {
+      tmem_st_x16(t_p, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(half_bar);
+    }
+  }
+  tmem_st_x16(t_p + 16, pk + 16);
+  const uint64_t q2 = fadd2(accq[0], accq[1]);
+  *qsum = f2_lo(q2) + f2_hi(q2);
+  const uint64_t e2 = fadd2(acc[0], acc[1]);
+  return f2_lo(e2) + f2_hi(e2);
+}
+
 // x rounded to the 16-bit MMA type and back.
 template <bool BF16>
 __device__ __forceinline__ float round16(float x) {
@@ -560,10 +637,13 @@ __device__ __forceinline__ float round16(float x) {
   else return __half2float(__float2half_rn(x));
 }
 
-template <int D, bool BF16, bool BIAS>
+template <int D, bool BF16, int MODE>
 __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uint32_t tmem,
                              const Ctl& c, int t) {
-  using L = Layout<D, BIAS>;
+  using L = Layout<D, MODE>;
+  constexpr bool BIAS = L::BIAS, FP8 = L::FP8;
+  (void)BIAS;
+  (void)FP8;
   const int r = threadIdx.x & 127;                           // row within the Q tile
   const uint32_t lane_base = (uint32_t)((threadIdx.x >> 5) & 3) * 32;
   const uint32_t t_s = tmem + (lane_base << 16) + S_COL[t];  // this warp's lanes of S_t / P_t
@@ -627,13 +707,22 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
       m = m_new;
       const float mref = (m == -INFINITY) ? 0.f : m;
       const uint32_t half_bar = bar_addr(sbase, BAR_PHALF + t);
-      const float lsum = masked ? exp_store<BF16, true>(s, sl2, mref, t_s, half_bar)
-                                : exp_store<BF16, false>(s, sl2, mref, t_s, half_bar);
-      const float pmax = ex2_approx(m_cand - mref);  // this tile's largest P
-      const float delta = round16<BF16>(pmax) - pmax;
-      tmem_wait_st();
-      l_e = l_e * alpha + lsum;
-      l_o = l_o * alpha + (lsum + delta);
+      if constexpr (FP8) {
+        float qsum;
+        const float lsum = masked ? exp_store_f8<true>(s, sl2, mref, t_s, half_bar, &qsum)
+                                  : exp_store_f8<false>(s, sl2, mref, t_s, half_bar, &qsum);
+        tmem_wait_st();
+        l_e = l_e * alpha + lsum;
+        l_o = l_o * alpha + qsum;
+      } else {
+        const float lsum = masked ? exp_store<BF16, true>(s, sl2, mref, t_s, half_bar)
+                                  : exp_store<BF16, false>(s, sl2, mref, t_s, half_bar);
+        const float pmax = ex2_approx(m_cand - mref);  // this tile's largest P
+        const float delta = round16<BF16>(pmax) - pmax;
+        tmem_wait_st();
+        l_e = l_e * alpha + lsum;
+        l_o = l_o * alpha + (lsum + delta);
+      }
       tc_fence_before();
       mbar_arrive(bar_addr(sbase, BAR_PFULL + t));
     }
@@ -659,10 +748,13 @@ __device__ __forceinline__ uint32_t cvt2(float lo, float hi) {
   }
 }
 
-template <int D, bool BF16, bool BIAS>
+template <int D, bool BF16, int MODE>
 __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, uint32_t tmem,
                                 const Ctl& c, const CUtensorMap* tm_o) {
-  using L = Layout<D, BIAS>;
+  using L = Layout<D, MODE>;
+  constexpr bool BIAS = L::BIAS, FP8 = L::FP8;
+  (void)BIAS;
+  (void)FP8;
   const int r = threadIdx.x & 127;
   const int wl = (threadIdx.x >> 5) & 3;  // warp within the group = 32-row slab
   const int lane = threadIdx.x & 31;
@@ -719,6 +811,7 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
         tc_fence_after();
         if (ml.y > 0.f) {
           inv_l = __frcp_rn(ml.y);
+          if constexpr (FP8) inv_l *= p.o_scale;
           lse = (ml.x + __log2f(ml.z)) * 0.69314718055994531f;
         }
       }
@@ -799,12 +892,15 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
 }
 
 // ================================================================== kernel
-template <int D, bool BF16, bool BIAS>
+template <int D, bool BF16, int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                   const __grid_constant__ CUtensorMap tm_b, const Params p) {
-  using L = Layout<D, BIAS>;
+  using L = Layout<D, MODE>;
+  constexpr bool BIAS = L::BIAS, FP8 = L::FP8;
+  (void)BIAS;
+  (void)FP8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -857,14 +953,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // Register split: 2×176 (softmax) + 80 (correction) + 80 (MMA, loads) = 4 × 128.
   if (warp < 8) {
     setmaxnreg_inc<176>();
-    role_softmax<D, BF16, BIAS>(p, smem, sbase, tmem, ctl, warp >> 2);
+    role_softmax<D, BF16, MODE>(p, smem, sbase, tmem, ctl, warp >> 2);
   } else if (warp < 12) {
     setmaxnreg_dec<80>();
-    role_correction<D, BF16, BIAS>(p, smem, sbase, tmem, ctl, &tm_o);
+    role_correction<D, BF16, MODE>(p, smem, sbase, tmem, ctl, &tm_o);
   } else {
     setmaxnreg_dec<80>();
-    if (warp == 12) role_mma<D, BF16, BIAS>(p, sbase, tmem, ctl);
-    if (warp == 13 && lane == 0) role_load<D, BIAS>(p, sbase, ctl, &tm_q, &tm_k, &tm_v);
+    if (warp == 12) role_mma<D, BF16, MODE>(p, sbase, tmem, ctl);
+    if (warp == 13 && lane == 0) role_load<D, MODE>(p, sbase, ctl, &tm_q, &tm_k, &tm_v);
     if constexpr (BIAS) {
       if (warp >= 14 && lane == 0) role_bias_load<D>(p, sbase, ctl, &tm_b, warp - 14);
     }
@@ -946,6 +1042,26 @@ __global__ void __launch_bounds__(256) fa_merge_splits_kernel(const float* __res
   }
 }
 
+// FP8 mode: V [BH][N][D] bytes -> Vᵀ [BH][D][N], so that the P·V product can
+// take V as a K-major operand. 64×64-byte tiles through shared memory.
+__global__ void __launch_bounds__(256) fa_transpose_u8_kernel(const uint8_t* __restrict__ v,
+                                                              uint8_t* __restrict__ vt, int N, int Dm) {
+  __shared__ uint8_t tile[64][65];
+  const long long bh = blockIdx.z;
+  const int n0 = blockIdx.x * 64, d0 = blockIdx.y * 64;
+  const uint8_t* src = v + bh * (long long)N * Dm;
+  uint8_t* dst = vt + bh * (long long)N * Dm;
+  for (int i = threadIdx.x; i < 64 * 64; i += blockDim.x) {
+    const int r = i / 64, cidx = i % 64;  // r: key, cidx: d
+    if (n0 + r < N) tile[r][cidx] = src[(long long)(n0 + r) * Dm + d0 + cidx];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 64 * 64; i += blockDim.x) {
+    const int r = i / 64, cidx = i % 64;  // r: d, cidx: key
+    if (n0 + cidx < N) dst[(long long)(d0 + r) * N + n0 + cidx] = tile[cidx][r];
+  }
+}
+
 // Evaluates the FMA-pipe exponential and ex2.approx on n inputs.
 __global__ void fa_exp2_selftest_kernel(const float* x, float* y_fma, float* y_mufu, int n) {
   const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
@@ -1017,7 +1133,7 @@ struct DeviceInfo {
   bool init = false;
   bool sm100 = false;
   int sms = 0;
-  bool attr_set[8] = {false, false, false, false, false, false, false, false};
+  bool attr_set[9] = {false, false, false, false, false, false, false, false, false};
   bool bwd_attr_set[4] = {false, false, false, false};
 };
 DeviceInfo g_dev[64];
@@ -1062,12 +1178,26 @@ int make_map(CUtensorMap* map, const void* ptr, bool bf16, int d, int n, long lo
   return FA_OK;
 }
 
-template <int D, bool BF16, bool BIAS = false>
+// 3-D map of bytes [heads][rows][inner] with 128×128-byte boxes, 128-byte swizzle.
+int make_map_u8(CUtensorMap* map, const void* ptr, int inner, int rows, long long heads) {
+  const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)heads};
+  const cuuint64_t strides[2] = {(cuuint64_t)inner, (cuuint64_t)inner * (cuuint64_t)rows};
+  const cuuint32_t box[3] = {128, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = driver_fns().encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr),
+                                   dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled (u8) failed (%d)", (int)r);
+  return FA_OK;
+}
+
+template <int D, bool BF16, int MODE = 0>
 int launch(const void* q, const void* k, const void* v, void* o, const fa::Params& prm,
            cudaStream_t stream, DeviceInfo& info, int slot, float* final_lse,
            const void* bias = nullptr, long long bias_planes = 0) {
-  using L = fa::Layout<D, BIAS>;
-  auto kern = fa::fa_fwd_kernel<D, BF16, BIAS>;
+  using L = fa::Layout<D, MODE>;
+  auto kern = fa::fa_fwd_kernel<D, BF16, MODE>;
   {
     std::lock_guard<std::mutex> lk(g_dev_mu);
     if (!info.attr_set[slot]) {
@@ -1088,18 +1218,26 @@ int launch(const void* q, const void* k, const void* v, void* o, const fa::Param
   CUtensorMap tq, tk, tv, to;
   const fa::Shape& s = prm.s;
   int rc;
-  if ((rc = make_map(&tq, q, BF16, D, s.N, (long long)s.B * s.Hq, 64, fa::BM,
-                     CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
-  if ((rc = make_map(&tk, k, BF16, D, s.N, (long long)s.B * s.Hk, 64, fa::BN,
-                     CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
-  if ((rc = make_map(&tv, v, BF16, D, s.N, (long long)s.B * s.Hk, 64, fa::BN,
-                     CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
+  if (MODE == 2) {
+    // E4M3 bytes: Q, K [heads][N][D] in 128×128-byte boxes; v is the transposed
+    // copy Vᵀ [heads][D][N] (row stride N bytes, a multiple of 16)
+    if ((rc = make_map_u8(&tq, q, D, s.N, (long long)s.B * s.Hq)) != FA_OK) return rc;
+    if ((rc = make_map_u8(&tk, k, D, s.N, (long long)s.B * s.Hk)) != FA_OK) return rc;
+    if ((rc = make_map_u8(&tv, v, s.N, D, (long long)s.B * s.Hk)) != FA_OK) return rc;
+  } else {
+    if ((rc = make_map(&tq, q, BF16, D, s.N, (long long)s.B * s.Hq, 64, fa::BM,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
+    if ((rc = make_map(&tk, k, BF16, D, s.N, (long long)s.B * s.Hk, 64, fa::BN,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
+    if ((rc = make_map(&tv, v, BF16, D, s.N, (long long)s.B * s.Hk, 64, fa::BN,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
+  }
   if ((rc = make_map(&to, o, BF16, D, s.N, (long long)s.B * s.Hq, 32, 32,
                      CU_TENSOR_MAP_SWIZZLE_64B)) != FA_OK) return rc;
   CUtensorMap tb;
   memset(&tb, 0, sizeof(tb));
   // bias planes [planes][N][N]: boxes of 64 keys × 128 query rows
-  if (BIAS && (rc = make_map(&tb, bias, BF16, s.N, s.N, bias_planes, 64, fa::BM,
+  if (MODE == 1 && (rc = make_map(&tb, bias, BF16, s.N, s.N, bias_planes, 64, fa::BM,
                              CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return rc;
   const int grid = s.num_units < info.sms ? s.num_units : info.sms;
   kern<<<grid, fa::NUM_THREADS, L::ALLOC, stream>>>(tq, tk, tv, to, tb, prm);
@@ -1263,6 +1401,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   prm.lse = lse;
   prm.o_part = nullptr;
   prm.lse_part = nullptr;
+  prm.o_scale = 1.f;
   prm.bias_bmul = bias_B > 1 ? 1 : 0;
   prm.bias_hmul = bias_H > 1 ? 1 : 0;
   prm.bias_H = bias_H > 0 ? bias_H : 1;
@@ -1292,10 +1431,10 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (bias != nullptr) {
     const long long planes = (long long)bias_B * bias_H;
     if (d == 128)
-      return bf16 ? launch<128, true, true>(q, k, v, o, prm, st, info, 4, lse, bias, planes)
-                  : launch<128, false, true>(q, k, v, o, prm, st, info, 5, lse, bias, planes);
-    return bf16 ? launch<64, true, true>(q, k, v, o, prm, st, info, 6, lse, bias, planes)
-                : launch<64, false, true>(q, k, v, o, prm, st, info, 7, lse, bias, planes);
+      return bf16 ? launch<128, true, 1>(q, k, v, o, prm, st, info, 4, lse, bias, planes)
+                  : launch<128, false, 1>(q, k, v, o, prm, st, info, 5, lse, bias, planes);
+    return bf16 ? launch<64, true, 1>(q, k, v, o, prm, st, info, 6, lse, bias, planes)
+                : launch<64, false, 1>(q, k, v, o, prm, st, info, 7, lse, bias, planes);
   }
   if (d == 128)
     return bf16 ? launch<128, true>(q, k, v, o, prm, st, info, 0, lse)
@@ -1482,6 +1621,7 @@ extern "C" int fa_fwd_splitkv_static(const void* q, const void* k, const void* v
   prm.lse = lse;
   prm.o_part = nullptr;
   prm.lse_part = nullptr;
+  prm.o_scale = 1.f;
   prm.bias_bmul = 0;
   prm.bias_hmul = 0;
   prm.bias_H = 1;
@@ -1687,4 +1827,103 @@ extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o
                 : bwd_launch<128, false>(q, k, v, o, lse, dout, dq, dk, dv, bp, dqacc, lse2, dsum, st, info, 1);
   return bf16 ? bwd_launch<64, true>(q, k, v, o, lse, dout, dq, dk, dv, bp, dqacc, lse2, dsum, st, info, 2)
               : bwd_launch<64, false>(q, k, v, o, lse, dout, dq, dk, dv, bp, dqacc, lse2, dsum, st, info, 3);
+}
+
+// ============================================================= FP8 forward
+namespace {
+size_t fp8_ws_bytes(long long heads_k, int N, int d) {
+  return ((size_t)heads_k * N * d + 255) / 256 * 256;
+}
+}  // namespace
+
+extern "C" size_t fa_fwd_fp8_workspace_bytes(int B, int Hk, int N, int d) {
+  if (B < 1 || Hk < 1 || N < 1 || d != 128) return 0;
+  return fp8_ws_bytes((long long)B * Hk, N, d);
+}
+
+extern "C" int fa_fwd_fp8(const void* q, const void* k, const void* v, float q_descale,
+                          float k_descale, float v_descale, void* o, float* lse, int B, int Hq,
+                          int Hk, int N, int d, float scale, int causal,
+                          const int32_t* key_pad_lens, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  g_err[0] = '\0';
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr)
+    return fail(FA_ERR_INVALID_ARG, "q, k, v and o must be non-NULL");
+  if (B < 1 || Hq < 1 || Hk < 1 || N < 1)
+    return fail(FA_ERR_INVALID_ARG, "B, Hq, Hk and N must be >= 1");
+  if (Hq % Hk != 0) return fail(FA_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hk (%d)", Hq, Hk);
+  if (d != 128) return fail(FA_ERR_UNSUPPORTED, "FP8 forward supports head dim 128, not %d", d);
+  if (N % 16 != 0)
+    return fail(FA_ERR_UNSUPPORTED, "FP8 forward needs N %% 16 == 0 (16-byte rows of Vᵀ), N = %d", N);
+  if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "scale must be finite");
+  if (!(std::isfinite(q_descale) && std::isfinite(k_descale) && std::isfinite(v_descale)) ||
+      q_descale <= 0.f || k_descale <= 0.f || v_descale <= 0.f)
+    return fail(FA_ERR_INVALID_ARG, "descale factors must be finite and > 0");
+  if (causal != 0 && causal != 1) return fail(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  const long long heads_q = (long long)B * Hq, heads_k = (long long)B * Hk;
+  if (heads_q > 0x7fffffffLL || N > (1 << 30))
+    return fail(FA_ERR_INVALID_ARG, "problem too large for 32-bit tile coordinates");
+  if (fa_num_units(B, Hq, Hk, N, causal) < 0) return FA_ERR_INVALID_ARG;
+  const size_t need = fp8_ws_bytes(heads_k, N, d);
+  if (workspace_bytes < need)
+    return fail(FA_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", workspace_bytes, need);
+  if (!driver_fns().ok) return fail(FA_ERR_CUDA, "CUDA driver entry points unavailable");
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return fail(FA_ERR_CUDA, "no current CUDA device");
+  DeviceInfo& info = g_dev[dev];
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!info.init) {
+      cudaDeviceProp prop;
+      if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess)
+        return fail(FA_ERR_CUDA, "cudaGetDeviceProperties failed");
+      info.sm100 = prop.major == 10 && prop.minor == 0;
+      info.sms = prop.multiProcessorCount;
+      info.init = true;
+    }
+  }
+  if (!info.sm100) return fail(FA_ERR_UNSUPPORTED, "device %d is not sm_100", dev);
+  const size_t q_bytes = (size_t)heads_q * N * d, kv_bytes = (size_t)heads_k * N * d;
+  const size_t o_bytes = q_bytes * 2, lse_bytes = (size_t)heads_q * N * 4;
+  int rc;
+  if ((rc = check_range("q", q, q_bytes, 16)) != FA_OK) return rc;
+  if ((rc = check_range("k", k, kv_bytes, 16)) != FA_OK) return rc;
+  if ((rc = check_range("v", v, kv_bytes, 16)) != FA_OK) return rc;
+  if ((rc = check_range("o", o, o_bytes, 16)) != FA_OK) return rc;
+  if (lse != nullptr && (rc = check_range("lse", lse, lse_bytes, 4)) != FA_OK) return rc;
+  if ((rc = check_range("workspace", workspace, need, 256)) != FA_OK) return rc;
+  if (key_pad_lens != nullptr &&
+      (rc = check_range("key_pad_lens", key_pad_lens, (size_t)B * 4, 4)) != FA_OK)
+    return rc;
+  struct Span { const void* p; size_t n; };
+  const Span outs[3] = {{o, o_bytes}, {lse, lse_bytes}, {workspace, need}};
+  const Span all[6] = {{q, q_bytes}, {k, kv_bytes}, {v, kv_bytes}, {o, o_bytes}, {lse, lse_bytes},
+                       {workspace, need}};
+  for (int i = 0; i < 3; ++i)
+    for (int j = 0; j < 6; ++j) {
+      if (j == 3 + i || outs[i].p == nullptr || all[j].p == nullptr) continue;
+      const uintptr_t a = reinterpret_cast<uintptr_t>(outs[i].p), b = reinterpret_cast<uintptr_t>(all[j].p);
+      if (a < b + all[j].n && b < a + outs[i].n)
+        return fail(FA_ERR_INVALID_ARG, "an output or the workspace overlaps another argument");
+    }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* vt = reinterpret_cast<uint8_t*>(workspace);
+  const dim3 tgrid((unsigned)((N + 63) / 64), (unsigned)(d / 64), (unsigned)heads_k);
+  fa::fa_transpose_u8_kernel<<<tgrid, 256, 0, st>>>(reinterpret_cast<const uint8_t*>(v), vt, N, d);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "V transpose launch: %s", cudaGetErrorString(e));
+  fa::Params prm;
+  prm.key_pad_lens = key_pad_lens;
+  prm.lse = lse;
+  prm.o_part = nullptr;
+  prm.lse_part = nullptr;
+  prm.o_scale = v_descale;
+  prm.bias_bmul = 0;
+  prm.bias_hmul = 0;
+  prm.bias_H = 1;
+  prm.s = fa::make_shape(B, Hq, Hk, N, causal, 1);
+  prm.scale_log2 = (float)((double)scale * q_descale * k_descale * 1.4426950408889634);
+  prm.timeout_ns = g_timeout_ns;
+  return launch<128, true, 2>(q, k, vt, o, prm, st, info, 8, lse);
 }
