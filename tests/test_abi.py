@@ -187,3 +187,34 @@ def test_bias_arguments_rejected_before_cuda():
     assert lib.fa_fwd_bias(*args(16, 1, 2, 64)) == -1 and "head" in binding.last_error()
     assert lib.fa_fwd_bias(*args(16, 2, 4, 60)) == -2 and "N % 8" in binding.last_error()
     assert lib.fa_fwd_bias(*args(None, 1, 1, 64)) == -1 and "NULL" in binding.last_error()
+
+
+def test_backward_arguments_rejected_before_cuda():
+    lib = binding.lib
+    args = lambda d, N, Hq=2, Hk=1, scale=0.1, causal=0, ws=1 << 30: (  # noqa: E731
+        16, 16, 16, 16, 16, 16, 16, 16, 16, 1, Hq, Hk, N, d, scale, causal, None, 16, ws, None, 1)
+    assert lib.fa_bwd(*args(96, 128)) == -2 and "head dim" in binding.last_error()
+    assert lib.fa_bwd(*args(128, 128, Hq=3, Hk=2)) == -1 and "multiple" in binding.last_error()
+    assert lib.fa_bwd(*args(128, 128, scale=float("nan"))) == -1
+    assert lib.fa_bwd(*args(128, 128, causal=2)) == -1
+    assert lib.fa_bwd(*args(128, 128, ws=0)) == -1 and "workspace" in binding.last_error()
+    nulls = (None,) + (16,) * 8 + (1, 2, 1, 128, 128, 0.1, 0, None, 16, 1 << 30, None, 1)
+    assert lib.fa_bwd(*nulls) == -1 and "NULL" in binding.last_error()
+    need = binding.lib.fa_bwd_workspace_bytes(2, 4, 300, 128)
+    npad = 384
+    rup = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert need == rup(8 * 300 * 128 * 4) + 2 * rup(8 * npad * 4)
+    assert binding.lib.fa_bwd_workspace_bytes(2, 4, 300, 80) == 0
+
+
+def test_fp8_arguments_rejected_before_cuda():
+    lib = binding.lib
+    args = lambda d, N, qs=1.0, ws=1 << 30: (16, 16, 16, qs, 1.0, 1.0, 16, None, 1, 2, 1, N, d,  # noqa: E731
+                                             0.1, 0, None, 16, ws, None)
+    assert lib.fa_fwd_fp8(*args(64, 128)) == -2 and "head dim" in binding.last_error()
+    assert lib.fa_fwd_fp8(*args(128, 100)) == -2 and "N % 16" in binding.last_error()
+    assert lib.fa_fwd_fp8(*args(128, 128, qs=0.0)) == -1 and "descale" in binding.last_error()
+    assert lib.fa_fwd_fp8(*args(128, 128, qs=float("inf"))) == -1
+    assert lib.fa_fwd_fp8(*args(128, 128, ws=0)) == -1 and "workspace" in binding.last_error()
+    assert binding.lib.fa_fwd_fp8_workspace_bytes(1, 2, 4096, 128) == 2 * 4096 * 128
+    assert binding.lib.fa_fwd_fp8_workspace_bytes(1, 2, 4096, 64) == 0
