@@ -38,7 +38,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0  # the same GEMM held under the 1 kW power cap
 KERNEL_SOURCES = ["tiled_online_softmax_03_b200/csrc/fa_fwd_sm100.cu",
                   "tiled_online_softmax_03_b200/csrc/fa_ptx.cuh",
-                  "tiled_online_softmax_03_b200/csrc/fa_schedule.cuh"]
+                  "tiled_online_softmax_03_b200/csrc/fa_schedule.cuh",
+                  "tiled_online_softmax_03_b200/csrc/fa_bwd_sm100.cuh"]
 
 
 def flops(w):
@@ -67,10 +68,11 @@ def peaks():
             "fallback (earlier measurement on this pool)"
 
 
-def recorded_traffic(workload):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
-    path = os.path.join(ROOT, "profiles", f"fa_fwd_{workload}.md")
+def recorded_traffic(workload, kind="fa_fwd"):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary profiles/<kind>_<workload>.md (kind: fa_fwd, fa_fwd_fp8, fa_bwd),
+    if it was taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kind}_{workload}.md")
     try:
         text = open(path, encoding="utf-8").read()
     except OSError:
@@ -528,8 +530,8 @@ def main():
     peak_src += ", sustained (sw_power_cap active in the timed region)" if peak == sustained and capped \
         else ", burst"
     achieved = f / (kern_avg * 1e-3) / 1e12
-    traffic = recorded_traffic(w.name) if (args.splits == 1 and args.bias == "none"
-                                           and not args.backward and not args.fp8) else None
+    kind = "fa_bwd" if args.backward else ("fa_fwd_fp8" if args.fp8 else "fa_fwd")
+    traffic = recorded_traffic(w.name, kind) if (args.splits == 1 and args.bias == "none") else None
     config = config_of(w, world)
     kernels = "fa_fwd_kernel"
     if args.splits > 1:
@@ -551,7 +553,9 @@ def main():
         "dtype": "e4m3" if f8 is not None else w.dtype, "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
         "config": config,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                     "frac": achieved / peak, "traffic": traffic,
+                     "traffic_of": "fa_bwd_kernel" if bwd is not None else "fa_fwd_kernel",
+                     "peak_source": peak_src,
                      "frac_of_burst": achieved / burst,
                      "kernel": kernels, "kernel_ms": kern_avg,
                      "flop_per_launch": f},

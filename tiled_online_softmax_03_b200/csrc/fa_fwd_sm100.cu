@@ -38,6 +38,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/fa.h"
 #include "fa_ptx.cuh"
@@ -125,7 +126,7 @@ struct Params {
 // UMMA shared-memory descriptor, sm_100 format: start address >> 4 in bits
 // 0-13, leading byte offset >> 4 in 16-29, stride byte offset >> 4 in 32-45,
 // version 1 in bit 46, layout (2 = 128-byte swizzle) in bits 61-63.
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+__host__ __device__ constexpr uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((addr & 0x3FFFF) >> 4) | ((uint64_t)(lbo >> 4) << 16) |
          ((uint64_t)(sbo >> 4) << 32) | (1ull << 46) | (2ull << 61);
 }
@@ -133,6 +134,30 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t 
 __host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int n, bool b_mn_major) {
   return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
          ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+// High word of every shared-memory descriptor used here (1024-byte stride
+// byte offset, version 1, 128-byte swizzle); only the low word varies.
+constexpr uint32_t SDESC_HI = (uint32_t)(sdesc(0, 16, 1024) >> 32);
+// Two spellings of the same MMAs: full 64-bit descriptors, or their low words
+// with SDESC_HI as a constant (fewer live registers in the issuing warp).
+template <bool F8>
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+  if constexpr (F8) umma_ss_f8_warp(d, a, b, id, acc);
+  else umma_ss_warp(d, a, b, id, acc);
+}
+template <bool F8>
+__device__ __forceinline__ void mma_ss(uint32_t d, uint32_t a, uint32_t b, uint32_t id, uint32_t acc) {
+  umma_ss_lo<F8, SDESC_HI, SDESC_HI>(d, a, b, id, acc);
+}
+template <bool F8>
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t id, uint32_t acc) {
+  if constexpr (F8) umma_ts_f8_warp(d, a_tmem, b, id, acc);
+  else umma_ts_warp(d, a_tmem, b, id, acc);
+}
+template <bool F8>
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint32_t b, uint32_t id, uint32_t acc) {
+  umma_ts_lo<F8, SDESC_HI>(d, a_tmem, b, id, acc);
 }
 
 // ------------------------------------------------------------ bounded waits
@@ -312,32 +337,36 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
   // once per call (a K step adds its byte offset >> 4 to the start-address
   // field, bits 0-13, with no carry out since shared memory is < 256 KB), and
   // the accumulate flag is a compile-time constant except on the first step.
-  const uint64_t q_desc0 = sdesc(sbase + L::OFF_Q, 16, 1024);
-  const uint64_t kv_desc0 = sdesc(sbase + L::OFF_KV, 16, 1024);
-  const uint64_t v_desc0 = FP8 ? sdesc(sbase + L::OFF_KV, 16, 1024)
-                                : sdesc(sbase + L::OFF_KV, SW128_BOX_BYTES, 1024);
+  // The plain kernels keep only the descriptors' low words live: the 64-bit
+  // form spilled in this 80-register warp and ran 4-5 % slower. The bias and
+  // FP8 kernels keep the 64-bit form (no spill in FP8; in the bias kernel the
+  // low-word form timed 13 % slower).
+  using Desc = std::conditional_t<MODE == 0, uint32_t, uint64_t>;
+  const Desc q_desc0 = (Desc)sdesc(sbase + L::OFF_Q, 16, 1024);
+  const Desc kv_desc0 = (Desc)sdesc(sbase + L::OFF_KV, 16, 1024);
+  const Desc v_desc0 = FP8 ? kv_desc0 : (Desc)sdesc(sbase + L::OFF_KV, SW128_BOX_BYTES, 1024);
   auto issue_qk = [&](int t, int kst) {
-    const uint64_t qd = q_desc0 + (uint64_t)((t * L::Q_BYTES) >> 4);
-    const uint64_t kd = kv_desc0 + (uint64_t)((kst * L::KV_BYTES) >> 4);
+    const Desc qd = q_desc0 + (Desc)((t * L::Q_BYTES) >> 4);
+    const Desc kd = kv_desc0 + (Desc)((kst * L::KV_BYTES) >> 4);
     const uint32_t d_s = tmem + S_COL[t];
     if constexpr (FP8) {  // K = 32 bytes per MMA, all inside one 128-byte row
-      umma_ss_f8_warp(d_s, qd, kd, IDESC_QK, 0u);
+      mma_ss<true>(d_s, qd, kd, IDESC_QK, 0u);
 #pragma unroll
-      for (int k = 1; k < D / 32; ++k) umma_ss_f8_warp(d_s, qd + 2 * k, kd + 2 * k, IDESC_QK, 1u);
+      for (int k = 1; k < D / 32; ++k) mma_ss<true>(d_s, qd + 2 * k, kd + 2 * k, IDESC_QK, 1u);
       return;
     }
-    umma_ss_warp(d_s, qd, kd, IDESC_QK, 0u);
+    mma_ss<false>(d_s, qd, kd, IDESC_QK, 0u);
 #pragma unroll
     for (int k = 1; k < D / 16; ++k) {
       const uint32_t off = ((k >> 2) * SW128_BOX_BYTES + (k & 3) * 32) >> 4;
-      umma_ss_warp(d_s, qd + off, kd + off, IDESC_QK, 1u);
+      mma_ss<false>(d_s, qd + off, kd + off, IDESC_QK, 1u);
     }
   };
   // P·V over keys [32·h, 32·h + 64) of the tile (h = 0: first half, 1: second).
   auto issue_pv_half = [&](int t, int vst, int h, uint32_t acc) {
     // P: 16 keys = 8 TMEM columns (two 16-bit values per column); V: 16 key
     // rows of 128 bytes in each 64-column box, boxes SW128_BOX_BYTES apart.
-    const uint64_t vd = v_desc0 + (uint64_t)((vst * L::KV_BYTES) >> 4);
+    const Desc vd = v_desc0 + (Desc)((vst * L::KV_BYTES) >> 4);
     const uint32_t d_o = tmem + TmemO<D>::col(t);
     const uint32_t a_p = tmem + S_COL[t];
     if constexpr (FP8) {
@@ -345,14 +374,14 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
       // hold keys, 32 keys = 32 bytes of each 128-byte row
 #pragma unroll
       for (int k = 2 * h; k < 2 * h + 2; ++k)
-        umma_ts_f8_warp(d_o, a_p + k * 8, vd + 2 * k, IDESC_PV, k == 0 ? acc : 1u);
+        mma_ts<true>(d_o, a_p + k * 8, vd + 2 * k, IDESC_PV, k == 0 ? acc : 1u);
       return;
     }
     const int k0 = h * (BN / 32);
-    umma_ts_warp(d_o, a_p + k0 * 8, vd + ((k0 * 16 * 128) >> 4), IDESC_PV, acc);
+    mma_ts<false>(d_o, a_p + k0 * 8, vd + ((k0 * 16 * 128) >> 4), IDESC_PV, acc);
 #pragma unroll
     for (int k = k0 + 1; k < k0 + BN / 32; ++k)
-      umma_ts_warp(d_o, a_p + k * 8, vd + ((k * 16 * 128) >> 4), IDESC_PV, 1u);
+      mma_ts<false>(d_o, a_p + k * 8, vd + ((k * 16 * 128) >> 4), IDESC_PV, 1u);
   };
 
   // Phase bits, one per barrier the MMA thread waits on.

@@ -186,6 +186,52 @@ __device__ __forceinline__ void umma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, u
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The same forms with each shared-memory descriptor passed as its low word
+// (start address >> 4, leading byte offset >> 4) and its high word (stride
+// byte offset, version, swizzle mode) as a compile-time constant, so that only
+// the low words occupy registers. F8 selects kind::f8f6f4 over kind::f16.
+template <bool F8, uint32_t A_HI, uint32_t B_HI>
+__device__ __forceinline__ void umma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                           uint32_t idesc, uint32_t accumulate) {
+  if constexpr (F8) {
+    asm volatile(
+        "{\n\t.reg .pred e, p;\n\t.reg .b64 a, b;\n\t"
+        "mov.b64 a, {%1, %5};\n\tmov.b64 b, {%2, %6};\n\t"
+        "elect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(A_HI), "r"(B_HI)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred e, p;\n\t.reg .b64 a, b;\n\t"
+        "mov.b64 a, {%1, %5};\n\tmov.b64 b, {%2, %6};\n\t"
+        "elect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(A_HI), "r"(B_HI)
+        : "memory");
+  }
+}
+template <bool F8, uint32_t B_HI>
+__device__ __forceinline__ void umma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                           uint32_t idesc, uint32_t accumulate) {
+  if constexpr (F8) {
+    asm volatile(
+        "{\n\t.reg .pred e, p;\n\t.reg .b64 b;\n\t"
+        "mov.b64 b, {%2, %5};\n\t"
+        "elect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], b, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(B_HI)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred e, p;\n\t.reg .b64 b;\n\t"
+        "mov.b64 b, {%2, %5};\n\t"
+        "elect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(B_HI)
+        : "memory");
+  }
+}
 // The same two MMA forms for 8-bit operands (kind::f8f6f4; K = 32 per
 // instruction; E4M3 is format 0 in the instruction descriptor's A/B fields).
 __device__ __forceinline__ void umma_ss_f8_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
