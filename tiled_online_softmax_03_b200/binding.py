@@ -148,6 +148,103 @@ def fa_fwd(q, k, v, causal=False, scale=None, key_pad_lens=None, out=None, lse=N
     return (out, lse) if return_lse else out
 
 
+_IO_STREAMS = {}
+
+
+def _io_streams(device):
+    """Two streams per device for the copies in and out of fa_fwd_from_host."""
+    key = device.index
+    if key not in _IO_STREAMS:
+        _IO_STREAMS[key] = (torch.cuda.Stream(device), torch.cuda.Stream(device))
+    return _IO_STREAMS[key]
+
+
+def fa_fwd_from_host(q, k, v, causal=False, scale=None, key_pad_lens=None, out=None, lse=None,
+                     device_buffers=None, device=None, stream=None):
+    """fa_fwd on page-locked HOST tensors, pipelined batch by batch.
+
+    q [B,Hq,N,d], k and v [B,Hk,N,d] (and key_pad_lens, int32 [B], if given)
+    are contiguous pinned CPU tensors; ``out`` [B,Hq,N,d] and ``lse``
+    [B,Hq,N] float32, pinned CPU tensors, receive the result (allocated pinned
+    when None). The device copies live in ``device_buffers``, a dict of CUDA
+    tensors 'q', 'k', 'v', 'o', 'lse' of the same shapes and, with padding,
+    'lens' [B] int32; they are allocated on ``device`` (default: the current
+    CUDA device) when None. For each batch b the copy in of batch b + 1, the
+    attention of batch b (one fa_fwd call of the C ABI on the batch's slices)
+    and the copy out of batch b − 1 run on three streams, so the two PCIe
+    directions and the kernel overlap. The kernels go on ``stream`` (a
+    torch.cuda.Stream; default the current stream), which on return is ordered
+    after every copy: synchronising it makes ``out`` and ``lse`` valid.
+    Consecutive calls on one stream do not overlap each other. Caller-given
+    device buffers must stay alive until then. Returns (out, lse).
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.is_cuda or not t.is_contiguous() or t.dim() != 4 or not t.is_pinned():
+            raise FaError(FA_ERR_INVALID_ARG, f"{name} must be a contiguous 4-D pinned CPU tensor")
+    if q.dtype not in _DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise FaError(FA_ERR_UNSUPPORTED, "q, k, v must share one dtype: float16 or bfloat16")
+    B, Hq, N, d = q.shape
+    Hk = k.shape[1]
+    if tuple(k.shape) != (B, Hk, N, d) or tuple(v.shape) != (B, Hk, N, d):
+        raise FaError(FA_ERR_INVALID_ARG, "k and v must be [B, Hk, N, d] matching q")
+    if key_pad_lens is not None and (key_pad_lens.is_cuda or key_pad_lens.dtype != torch.int32 or
+                                     key_pad_lens.numel() != B or not key_pad_lens.is_pinned()):
+        raise FaError(FA_ERR_INVALID_ARG, "key_pad_lens must be a pinned int32 CPU tensor [B]")
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32).pin_memory()
+    if out.is_cuda or tuple(out.shape) != tuple(q.shape) or out.dtype != q.dtype or \
+            not out.is_contiguous() or not out.is_pinned():
+        raise FaError(FA_ERR_INVALID_ARG, "out must be a pinned CPU tensor shaped and typed like q")
+    if lse.is_cuda or tuple(lse.shape) != (B, Hq, N) or lse.dtype != torch.float32 or \
+            not lse.is_contiguous() or not lse.is_pinned():
+        raise FaError(FA_ERR_INVALID_ARG, "lse must be a pinned float32 CPU tensor [B, Hq, N]")
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    cs = torch.cuda.current_stream(device) if stream is None else stream
+    s_in, s_out = _io_streams(device)
+    owned = device_buffers is None
+    if owned:
+        device_buffers = {"q": torch.empty(q.shape, dtype=q.dtype, device=device),
+                          "k": torch.empty(k.shape, dtype=q.dtype, device=device),
+                          "v": torch.empty(v.shape, dtype=q.dtype, device=device),
+                          "o": torch.empty(q.shape, dtype=q.dtype, device=device),
+                          "lse": torch.empty((B, Hq, N), dtype=torch.float32, device=device),
+                          "lens": (torch.empty(B, dtype=torch.int32, device=device)
+                                   if key_pad_lens is not None else None)}
+    qd, kd, vd, od, ld = (device_buffers[n] for n in ("q", "k", "v", "o", "lse"))
+    lens_d = device_buffers.get("lens") if key_pad_lens is not None else None
+    if key_pad_lens is not None and lens_d is None:
+        raise FaError(FA_ERR_INVALID_ARG, "device_buffers needs 'lens' when key_pad_lens is given")
+    if owned:
+        for t in (qd, kd, vd, od, ld) + ((lens_d,) if lens_d is not None else ()):
+            t.record_stream(s_in)
+            t.record_stream(s_out)
+    # earlier work on the stream, the previous call's copies out included,
+    # comes first: the device buffers are reused
+    cs.wait_stream(s_out)
+    s_in.wait_stream(cs)
+    s_out.wait_stream(cs)
+    if lens_d is not None:
+        with torch.cuda.stream(s_in):
+            lens_d.copy_(key_pad_lens, non_blocking=True)
+    for b in range(B):
+        with torch.cuda.stream(s_in):
+            qd[b].copy_(q[b], non_blocking=True)
+            kd[b].copy_(k[b], non_blocking=True)
+            vd[b].copy_(v[b], non_blocking=True)
+        cs.wait_event(s_in.record_event())
+        fa_fwd(qd[b:b + 1], kd[b:b + 1], vd[b:b + 1], causal=causal, scale=scale,
+               key_pad_lens=lens_d[b:b + 1] if lens_d is not None else None,
+               out=od[b:b + 1], lse=ld[b:b + 1], stream=cs.cuda_stream)
+        s_out.wait_event(cs.record_event())
+        with torch.cuda.stream(s_out):
+            out[b].copy_(od[b], non_blocking=True)
+            lse[b].copy_(ld[b], non_blocking=True)
+    cs.wait_stream(s_out)
+    return out, lse
+
+
 def fa_fwd_bias(q, k, v, bias, causal=False, scale=None, key_pad_lens=None, out=None, lse=None,
                 return_lse=True, stream=None):
     """``fa_fwd`` with an additive bias on the scaled scores.
