@@ -576,7 +576,7 @@ def main():
         "e2e": {"value": whole_job_tflops(f, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "steps": e2e_steps,
-                "path": "fa_fwd_from_host (per-batch copy/attention/copy pipeline)" if pipelined
+                "path": "fa_fwd_from_host (per-chunk copy/attention/copy pipeline)" if pipelined
                 else "copies in, the call, copies out on one stream",
                 "matches_device_run": e2e_same},
         "gpu_launches": args.steps * (3 if bwd is not None else 2 if (args.splits > 1 or f8 is not None)

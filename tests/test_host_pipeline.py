@@ -47,6 +47,33 @@ def test_equals_device_call_bitwise(B, Hq, Hk, N, d, dtype, causal, lens):
     assert torch.equal(o, o_ref.cpu()) and torch.equal(lse, l_ref.cpu())
 
 
+@pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 6, 31, 32, 33])
+@pytest.mark.parametrize("chunks", [None, 1, 2, 3, 100])
+def test_chunk_ranges_partition_the_batch(B, chunks):
+    from tiled_online_softmax_03_b200.binding import chunk_ranges
+    r = chunk_ranges(B, chunks)
+    assert r[0][0] == 0 and r[-1][1] == B
+    assert all(a1 == b0 for (_, a1), (b0, _) in zip(r, r[1:]))
+    sizes = [b1 - b0 for b0, b1 in r]
+    assert min(sizes) >= 1 and max(sizes) - min(sizes) <= 1
+    assert len(r) == (min(B, 4) if chunks is None else min(chunks, B))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("chunks", [None, 1, 3, 6])
+def test_multi_batch_chunks_equal_device_call(chunks):
+    from tiled_online_softmax_03_b200 import binding
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    B, Hq, Hk, N, d = 6, 4, 2, 200, 64
+    w, x, L = _host_inputs(B, Hq, Hk, N, d, "bf16", False, [200, 0, 7, 128, 129, 55], seed=11)
+    dev = torch.device("cuda:0")
+    o_ref, l_ref = binding.fa_fwd(x["q"].to(dev), x["k"].to(dev), x["v"].to(dev), key_pad_lens=L.to(dev))
+    hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
+    o, lse = binding.fa_fwd_from_host(hq, hk, hv, key_pad_lens=L.pin_memory(), chunks=chunks)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref.cpu()) and torch.equal(lse, l_ref.cpu())
+
+
 @pytest.mark.gpu
 def test_reused_buffers_across_calls():
     """Two calls in a row on one stream with the same device buffers and new
@@ -70,3 +97,76 @@ def test_reused_buffers_across_calls():
     for x, o, lse in results:
         o_ref, l_ref = binding.fa_fwd(x["q"].to(dev), x["k"].to(dev), x["v"].to(dev), causal=True)
         assert torch.equal(o, o_ref.cpu()) and torch.equal(lse, l_ref.cpu())
+
+
+class _FakeDev:
+    """Stands in for a CUDA tensor in the host-side argument checks."""
+
+    def __init__(self, shape, dtype, device="cuda:0", contiguous=True):
+        self.shape = tuple(shape)
+        self.dtype = dtype
+        self.device = torch.device(device)
+        self.is_cuda = self.device.type == "cuda"
+        self._c = contiguous
+
+    def is_contiguous(self):
+        return self._c
+
+
+class _Pinned:
+    """A CPU tensor that reports itself page-locked (no CUDA on this host)."""
+
+    def __init__(self, t):
+        self.t = t
+        self.shape, self.dtype, self.is_cuda = t.shape, t.dtype, False
+
+    def __getattr__(self, name):
+        return getattr(self.t, name)
+
+    def is_pinned(self):
+        return True
+
+    def dim(self):
+        return self.t.dim()
+
+    def numel(self):
+        return self.t.numel()
+
+    def is_contiguous(self):
+        return True
+
+
+def _buffers(B, Hq, Hk, N, d, dt, lens=True, **override):
+    bufs = {"q": _FakeDev((B, Hq, N, d), dt), "k": _FakeDev((B, Hk, N, d), dt),
+            "v": _FakeDev((B, Hk, N, d), dt), "o": _FakeDev((B, Hq, N, d), dt),
+            "lse": _FakeDev((B, Hq, N), torch.float32),
+            "lens": _FakeDev((B,), torch.int32) if lens else None}
+    bufs.update(override)
+    return bufs
+
+
+@pytest.mark.parametrize("bad", [
+    {"o": _FakeDev((2, 4, 100, 64), torch.float16)},              # wrong head count
+    {"lse": _FakeDev((2, 2, 100), torch.float16)},                # wrong dtype
+    {"k": _FakeDev((2, 1, 100, 64), torch.bfloat16, "cuda:1")},   # other device
+    {"v": _FakeDev((2, 1, 100, 64), torch.bfloat16, contiguous=False)},
+    {"lens": None},                                              # padding without a buffer
+])
+def test_device_buffer_checks(bad):
+    from tiled_online_softmax_03_b200 import binding
+    B, Hq, Hk, N, d = 2, 2, 1, 100, 64
+    dt = torch.bfloat16
+    q, k, v = (_Pinned(torch.zeros(s, dtype=dt)) for s in [(B, Hq, N, d), (B, Hk, N, d), (B, Hk, N, d)])
+    out, lse = _Pinned(torch.zeros((B, Hq, N, d), dtype=dt)), _Pinned(torch.zeros((B, Hq, N)))
+    lens = _Pinned(torch.zeros(B, dtype=torch.int32))
+    with pytest.raises(binding.FaError, match="device_buffers"):
+        binding.fa_fwd_from_host(q, k, v, key_pad_lens=lens, out=out, lse=lse,
+                                 device_buffers=_buffers(B, Hq, Hk, N, d, dt, **bad),
+                                 device=torch.device("cuda", 0))
+    # the buffers the benchmark passes get past every check (up to the first
+    # CUDA call, which this host cannot make)
+    with pytest.raises(Exception) as e:
+        binding.fa_fwd_from_host(q, k, v, key_pad_lens=lens, out=out, lse=lse,
+                                 device_buffers=_buffers(B, Hq, Hk, N, d, dt),
+                                 device=torch.device("cuda", 0))
+    assert not isinstance(e.value, binding.FaError), e.value

@@ -160,8 +160,8 @@ def _io_streams(device):
 
 
 def fa_fwd_from_host(q, k, v, causal=False, scale=None, key_pad_lens=None, out=None, lse=None,
-                     device_buffers=None, device=None, stream=None):
-    """fa_fwd on page-locked HOST tensors, pipelined batch by batch.
+                     device_buffers=None, device=None, stream=None, chunks=None):
+    """fa_fwd on page-locked HOST tensors, pipelined chunk by chunk of the batch.
 
     q [B,Hq,N,d], k and v [B,Hk,N,d] (and key_pad_lens, int32 [B], if given)
     are contiguous pinned CPU tensors; ``out`` [B,Hq,N,d] and ``lse``
@@ -169,10 +169,12 @@ def fa_fwd_from_host(q, k, v, causal=False, scale=None, key_pad_lens=None, out=N
     when None). The device copies live in ``device_buffers``, a dict of CUDA
     tensors 'q', 'k', 'v', 'o', 'lse' of the same shapes and, with padding,
     'lens' [B] int32; they are allocated on ``device`` (default: the current
-    CUDA device) when None. For each batch b the copy in of batch b + 1, the
-    attention of batch b (one fa_fwd call of the C ABI on the batch's slices)
-    and the copy out of batch b − 1 run on three streams, so the two PCIe
-    directions and the kernel overlap. The kernels go on ``stream`` (a
+    CUDA device) when None. The batch is cut into ``chunks`` near-equal runs
+    of consecutive batches (default min(B, 4): large enough copies, and
+    launches that still fill the GPU); for each chunk c the copy in of chunk
+    c + 1, the attention of chunk c (one fa_fwd call of the C ABI on the
+    chunk's slices) and the copy out of chunk c − 1 run on three streams, so
+    the two PCIe directions and the kernel overlap. The kernels go on ``stream`` (a
     torch.cuda.Stream; default the current stream), which on return is ordered
     after every copy: synchronising it makes ``out`` and ``lse`` valid.
     Consecutive calls on one stream do not overlap each other. Caller-given
@@ -200,9 +202,14 @@ def fa_fwd_from_host(q, k, v, causal=False, scale=None, key_pad_lens=None, out=N
     if lse.is_cuda or tuple(lse.shape) != (B, Hq, N) or lse.dtype != torch.float32 or \
             not lse.is_contiguous() or not lse.is_pinned():
         raise FaError(FA_ERR_INVALID_ARG, "lse must be a pinned float32 CPU tensor [B, Hq, N]")
-    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
-    cs = torch.cuda.current_stream(device) if stream is None else stream
-    s_in, s_out = _io_streams(device)
+    if device is None:
+        device = device_buffers["q"].device if device_buffers is not None and "q" in device_buffers \
+            else torch.device("cuda", torch.cuda.current_device())
+    device = torch.device(device)
+    if device.type != "cuda":
+        raise FaError(FA_ERR_INVALID_ARG, "device must be a CUDA device")
+    if device.index is None:
+        device = torch.device("cuda", torch.cuda.current_device())
     owned = device_buffers is None
     if owned:
         device_buffers = {"q": torch.empty(q.shape, dtype=q.dtype, device=device),
@@ -212,10 +219,20 @@ def fa_fwd_from_host(q, k, v, causal=False, scale=None, key_pad_lens=None, out=N
                           "lse": torch.empty((B, Hq, N), dtype=torch.float32, device=device),
                           "lens": (torch.empty(B, dtype=torch.int32, device=device)
                                    if key_pad_lens is not None else None)}
+    want = {"q": (tuple(q.shape), q.dtype), "k": (tuple(k.shape), q.dtype), "v": (tuple(v.shape), q.dtype),
+            "o": (tuple(q.shape), q.dtype), "lse": ((B, Hq, N), torch.float32)}
+    if key_pad_lens is not None:
+        want["lens"] = ((B,), torch.int32)
+    for n, (shape, dt) in want.items():
+        t = device_buffers.get(n)
+        if t is None or not t.is_cuda or t.device != device or tuple(t.shape) != shape or \
+                t.dtype != dt or not t.is_contiguous():
+            raise FaError(FA_ERR_INVALID_ARG,
+                          f"device_buffers['{n}'] must be a contiguous {dt} tensor {list(shape)} on {device}")
     qd, kd, vd, od, ld = (device_buffers[n] for n in ("q", "k", "v", "o", "lse"))
-    lens_d = device_buffers.get("lens") if key_pad_lens is not None else None
-    if key_pad_lens is not None and lens_d is None:
-        raise FaError(FA_ERR_INVALID_ARG, "device_buffers needs 'lens' when key_pad_lens is given")
+    lens_d = device_buffers["lens"] if key_pad_lens is not None else None
+    cs = torch.cuda.current_stream(device) if stream is None else stream
+    s_in, s_out = _io_streams(device)
     if owned:
         for t in (qd, kd, vd, od, ld) + ((lens_d,) if lens_d is not None else ()):
             t.record_stream(s_in)
@@ -228,21 +245,34 @@ def fa_fwd_from_host(q, k, v, causal=False, scale=None, key_pad_lens=None, out=N
     if lens_d is not None:
         with torch.cuda.stream(s_in):
             lens_d.copy_(key_pad_lens, non_blocking=True)
-    for b in range(B):
+    for b0, b1 in chunk_ranges(B, chunks):
         with torch.cuda.stream(s_in):
-            qd[b].copy_(q[b], non_blocking=True)
-            kd[b].copy_(k[b], non_blocking=True)
-            vd[b].copy_(v[b], non_blocking=True)
+            qd[b0:b1].copy_(q[b0:b1], non_blocking=True)
+            kd[b0:b1].copy_(k[b0:b1], non_blocking=True)
+            vd[b0:b1].copy_(v[b0:b1], non_blocking=True)
         cs.wait_event(s_in.record_event())
-        fa_fwd(qd[b:b + 1], kd[b:b + 1], vd[b:b + 1], causal=causal, scale=scale,
-               key_pad_lens=lens_d[b:b + 1] if lens_d is not None else None,
-               out=od[b:b + 1], lse=ld[b:b + 1], stream=cs.cuda_stream)
+        fa_fwd(qd[b0:b1], kd[b0:b1], vd[b0:b1], causal=causal, scale=scale,
+               key_pad_lens=lens_d[b0:b1] if lens_d is not None else None,
+               out=od[b0:b1], lse=ld[b0:b1], stream=cs.cuda_stream)
         s_out.wait_event(cs.record_event())
         with torch.cuda.stream(s_out):
-            out[b].copy_(od[b], non_blocking=True)
-            lse[b].copy_(ld[b], non_blocking=True)
+            out[b0:b1].copy_(od[b0:b1], non_blocking=True)
+            lse[b0:b1].copy_(ld[b0:b1], non_blocking=True)
     cs.wait_stream(s_out)
     return out, lse
+
+
+def chunk_ranges(B, chunks=None):
+    """[b0, b1) runs of consecutive batches: ``chunks`` (default min(B, 4))
+    near-equal parts, the first B % chunks one batch longer."""
+    n = min(B, 4) if chunks is None else max(1, min(int(chunks), B))
+    base, extra = divmod(B, n)
+    out, b0 = [], 0
+    for i in range(n):
+        b1 = b0 + base + (1 if i < extra else 0)
+        out.append((b0, b1))
+        b0 = b1
+    return out
 
 
 def fa_fwd_bias(q, k, v, bias, causal=False, scale=None, key_pad_lens=None, out=None, lse=None,
