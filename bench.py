@@ -91,74 +91,128 @@ def recorded_traffic(workload, kind="fa_fwd"):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clock, power and throttle reasons sampled during the timed region.
+
+    Reads NVML (pynvml) from a thread every 5 ms, so that even a timed region
+    of a few tens of milliseconds holds several samples; falls back to
+    `nvidia-smi -lms 50` when NVML cannot be used. Read-only: no setting of
+    the GPU is changed."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, index):
+    def __init__(self, index, pci_bus_id=None, period_s=0.005):
         self.index = index
-        self.lines = []  # (host time received, csv line)
+        self.pci_bus_id = pci_bus_id
+        self.period_s = period_s
+        self.rows = []  # (host time, sm MHz, max MHz, power W, [reasons])
         self.proc = None
+        self.thread = None
         self.window = None
+        self.source = None
+        self._stop = threading.Event()
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.pci_bus_id:
+            try:
+                return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(self.pci_bus_id)
+            except pynvml.NVMLError:
+                pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _nvml_loop(self, nv, h):
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                r = int(get_reasons(h))
+                self.rows.append((time.time(), sm, mx, pw, [n for n, b in bits.items() if r & b]))
+            except nv.NVMLError:
+                pass
+            self._stop.wait(self.period_s)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            nv, h = self._nvml_handle()
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
             self.thread.start()
-        except OSError:
-            self.proc = None
+            self.source = "nvml, 5 ms period"
+        except Exception:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                     "--format=csv,noheader,nounits", "-lms", "50"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.thread = threading.Thread(target=self._smi_loop, daemon=True)
+                self.thread.start()
+                self.source = "nvidia-smi, 50 ms period"
+            except OSError:
+                self.proc = None
         time.sleep(0.3)
         return self
 
-    def _read(self):
+    @classmethod
+    def parse_smi(cls, t, line):
+        """(t, sm MHz, max MHz, power W, reasons) from one nvidia-smi csv line, or None."""
+        parts = [p.strip() for p in line.strip().split(",")]
+        if len(parts) < 9:
+            return None
+        try:
+            sm, mx, pw = float(parts[1]), float(parts[2]), float(parts[3])
+        except ValueError:
+            return None
+        return (t, sm, mx, pw, [n for n, f in zip(cls.NAMES, parts[5:9]) if f.lower() == "active"])
+
+    def _smi_loop(self):
         for line in self.proc.stdout:
-            self.lines.append((time.time(), line.strip()))
+            row = self.parse_smi(time.time(), line)
+            if row is not None:
+                self.rows.append(row)
 
     def mark(self, start, end):
         """Host times bracketing the timed region (after synchronising)."""
         self.window = (start, end)
 
     def __exit__(self, *exc):
+        time.sleep(0.05)
+        self._stop.set()
         if self.proc is not None:
-            time.sleep(0.15)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
     def summary(self):
         """Clocks, power and throttle reasons over the samples taken inside the
-        timed region (all samples if no region was marked)."""
-        rows = []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for t, line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                s, m = float(parts[1]), float(parts[2])
-                pw = float(parts[3])
-            except ValueError:
-                continue
-            rows.append((t, s, m, pw, [n for n, f in zip(names, parts[5:9]) if f.lower() == "active"]))
+        timed region (all samples if no region was marked or none fell in it)."""
+        rows = list(self.rows)
+        inside = rows
         if self.window is not None:
-            inside = [r for r in rows if self.window[0] <= r[0] <= self.window[1]]
-            rows = inside or rows
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        reasons = sorted({n for r in rows for n in r[4]})
-        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": rows[-1][2],
-                "sm_mhz_min": min(r[1] for r in rows),
-                "power_w_median": statistics.median(r[3] for r in rows),
-                "reasons": reasons, "samples": len(rows),
-                "window": "samples taken inside the timed region" if self.window else "all samples"}
+            inside = [r for r in rows if self.window[0] <= r[0] <= self.window[1]] or rows
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": self.source}
+        reasons = sorted({n for r in inside for n in r[4]})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": inside[-1][2],
+                "sm_mhz_min": min(r[1] for r in inside),
+                "power_w_median": statistics.median(r[3] for r in inside),
+                "reasons": reasons, "samples": len(inside), "source": self.source,
+                "window": "samples taken inside the timed region"
+                if self.window is not None and inside is not rows else "all samples"}
 
 
 class OracleSampler:
@@ -290,6 +344,92 @@ def in_bytes(w):
     return 2 * w.B * w.N * w.d * (w.Hq + 2 * w.Hk)
 
 
+def algorithmic_bytes(w):
+    """HBM bytes the method must move once: Q, K, V in, O and LSE (fp32) out."""
+    return in_bytes(w) + 2 * w.B * w.Hq * w.N * w.d + 4 * w.B * w.Hq * w.N
+
+
+def pci_bus_id(dev):
+    """NVML-style PCI bus id of a torch CUDA device, or None."""
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        return None
+
+
+# The workloads timed after the headline one (every shape the metric is quoted on).
+PER_WORKLOAD = ["gqa_8k_causal", "mqa_8k_causal", "long_32k_causal", "llama7b_4k_causal",
+                "bert_large_512_keypad", "single_head_128"]
+
+
+def time_forward(w, dev, stream, steps, warmup, rank, local, world, barrier, rank_max, binding):
+    """Times fa_fwd on workload w exactly as the headline loop does: warm-up
+    launches, then `steps` launches with CUDA events around each on the
+    launching stream, an L2 flush between launches when the inputs fit in L2
+    (only the launches' own event times then count), clocks sampled in the
+    timed region, max over ranks. Returns a summary dict."""
+    x = rank_inputs(w, rank)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    lens = x["key_pad_lens"].to(dev) if x["key_pad_lens"] is not None else None
+    o = torch.empty_like(q)
+    lse = torch.empty(w.B, w.Hq, w.N, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if in_bytes(w) <= 126e6 else None
+
+    def call():
+        binding.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, key_pad_lens=lens, out=o, lse=lse,
+                       stream=stream.cuda_stream)
+
+    for _ in range(warmup):
+        if flush is not None:
+            flush.fill_(1)
+        call()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local, pci_bus_id(dev)) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        host_t0 = time.time()
+        t_begin.record(stream)
+        for i in range(steps):
+            if flush is not None:
+                flush.fill_(1)
+            starts[i].record(stream)
+            call()
+            ends[i].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        clocks.mark(host_t0, time.time())
+        barrier()
+    status = binding.device_status()
+    kern = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    kern_avg = rank_max(sum(kern) / len(kern))
+    total = rank_max(t_begin.elapsed_time(t_end)) if flush is None else kern_avg * steps
+    del q, k, v, o, lse, flush
+    torch.cuda.empty_cache()
+    return {"kernel_ms": kern_avg, "kernel_ms_median": rank_max(statistics.median(kern)),
+            "ms_per_step": total / steps, "clocks": clocks.summary(), "device_status": status,
+            "l2": "inputs larger than L2 (no flush)" if in_bytes(w) > 126e6 else
+                  "L2 flushed between steps (256 MB write); kernel event times only"}
+
+
+def workload_entry(w, t, world, burst, sustained):
+    """One per_workload record: whole-job TFLOP/s, roofline fractions, GB/s."""
+    f = flops(w)
+    achieved = f / (t["kernel_ms"] * 1e-3) / 1e12
+    return {"B": w.B, "Hq": w.Hq, "Hk": w.Hk, "N": w.N, "d": w.d, "causal": w.causal,
+            "key_pad": w.key_pad, "in_dtype": w.dtype,
+            "value": whole_job_tflops(f, world, t["ms_per_step"]), "unit": "TFLOP/s",
+            "kernel_ms": t["kernel_ms"], "kernel_ms_median": t["kernel_ms_median"],
+            "ms_per_step": t["ms_per_step"], "achieved_tflops": achieved,
+            "frac_of_burst": achieved / burst,
+            "frac_of_sustained": achieved / sustained if sustained else None,
+            "algorithmic_gbps": algorithmic_bytes(w) / (t["kernel_ms"] * 1e-3) / 1e9,
+            "clocks": t["clocks"], "l2": t["l2"], "device_status": t["device_status"]}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -307,6 +447,8 @@ def main():
                     help="time fa_fwd_fp8 on the workload's inputs quantised per tensor to E4M3")
     ap.add_argument("--backward", action="store_true",
                     help="time fa_bwd (dQ, dK, dV for a seeded dO) instead of the forward")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip timing the other workloads after the headline one")
     ap.add_argument("--splits", type=int, default=1,
                     help="K/V splits per Q tile pair (fa_fwd_splitkv; 1 = fa_fwd)")
     args = ap.parse_args()
@@ -424,7 +566,7 @@ def main():
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     t_begin = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clocks:
+    with ClockSampler(local, pci_bus_id(dev)) as clocks:
         barrier()
         torch.cuda.synchronize()
         host_t0 = time.time()
@@ -524,6 +666,17 @@ def main():
         h2d = sum(t.numel() * t.element_size() for t in hf8.values()) + \
             (hlens.numel() * 4 if hlens is not None else 0)
 
+    # ---- every other workload, timed the same way (plain forward runs only)
+    per_wl = {}
+    plain = pipelined and not args.shape and not args.no_per_workload
+    if plain:
+        del hq_, hk_, hv_, ho, hl
+        for name in PER_WORKLOAD:
+            if name == w.name:
+                continue
+            per_wl[name] = time_forward(WORKLOADS[name], dev, stream, args.steps, args.warmup,
+                                        rank, local, world, barrier, rank_max, binding)
+
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -584,6 +737,15 @@ def main():
         "clocks": clk,
         "device_status": status,
     }
+    if plain:
+        head = {"kernel_ms": kern_avg, "kernel_ms_median": statistics.median(kern_ms),
+                "ms_per_step": ms_per_step, "clocks": clk, "device_status": status,
+                "l2": config["l2"]}
+        line["per_workload"] = {name: workload_entry(WORKLOADS[name], head if name == w.name
+                                                     else per_wl[name], world, burst,
+                                                     sustained if f8 is None else None)
+                                for name in PER_WORKLOAD if name == w.name or name in per_wl}
+        line["gpu_launches_per_workload"] = args.steps
     if world == 1 and not args.no_cpu_baseline and bwd is None and f8 is None:
         line["cpu_baseline"] = {k2: v2 for k2, v2 in cpu_baseline(w).items()
                                 if k2 not in ("seconds", "heads")}

@@ -58,20 +58,32 @@ def test_kernel_hash_covers_every_kernel_source():
 def test_clock_summary_keeps_the_timed_window():
     c = bench.ClockSampler(0)
     line = "0, {sm}, 1965, {pw}, 0x0, {hw}, Not Active, Not Active, {cap}"
-    c.lines = [(1.0, line.format(sm=1965, pw=300, hw="Active", cap="Not Active")),    # before
-               (2.0, line.format(sm=1700, pw=990, hw="Not Active", cap="Active")),
-               (2.5, line.format(sm=1650, pw=1000, hw="Not Active", cap="Active")),
-               (3.0, line.format(sm=1680, pw=995, hw="Not Active", cap="Active")),
-               (4.0, line.format(sm=1965, pw=200, hw="Not Active", cap="Not Active"))]  # after
+    c.rows = [bench.ClockSampler.parse_smi(t, line.format(sm=sm, pw=pw, hw=hw, cap=cap))
+              for t, sm, pw, hw, cap in [
+                  (1.0, 1965, 300, "Active", "Not Active"),       # before the window
+                  (2.0, 1700, 990, "Not Active", "Active"),
+                  (2.5, 1650, 1000, "Not Active", "Active"),
+                  (3.0, 1680, 995, "Not Active", "Active"),
+                  (4.0, 1965, 200, "Not Active", "Not Active")]]  # after
     c.mark(1.5, 3.5)
     s = c.summary()
     assert s["samples"] == 3 and s["sm_mhz"] == 1680 and s["sm_mhz_min"] == 1650
     assert s["reasons"] == ["sw_power_cap"]  # the hw_slowdown sample lies outside the window
     assert s["sm_max_mhz"] == 1965 and s["power_w_median"] == 995
+    assert s["window"] == "samples taken inside the timed region"
 
 
 def test_clock_summary_without_samples():
     c = bench.ClockSampler(0)
-    c.lines = [(1.0, "garbage"), (1.5, "0, n/a, 1965, 1, 0x0, a, b, c, d")]
+    assert bench.ClockSampler.parse_smi(1.0, "garbage") is None
+    assert bench.ClockSampler.parse_smi(1.5, "0, n/a, 1965, 1, 0x0, a, b, c, d") is None
     s = c.summary()
     assert s["samples"] == 0 and s["sm_mhz"] is None and s["reasons"] == []
+
+
+def test_clock_summary_window_without_samples_uses_all():
+    c = bench.ClockSampler(0)
+    c.rows = [(1.0, 1965.0, 1965.0, 500.0, []), (5.0, 1900.0, 1965.0, 600.0, [])]
+    c.mark(2.0, 3.0)  # a region shorter than the sampling period
+    s = c.summary()
+    assert s["samples"] == 2 and s["window"] == "all samples"

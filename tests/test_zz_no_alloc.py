@@ -1,15 +1,22 @@
 """fa_fwd_splitkv_static: split-KV on the library's static scratch, no allocation.
 
+Some callers cannot allocate device memory per call: a server that reserved
+nearly all of HBM for weights and cache up front, a latency-critical loop in
+which cudaMalloc/cudaFree would synchronise the device, or a plain C caller
+with no memory pool. For them the library keeps its split-KV scratch in a
+fixed file-scope device array and this entry point only takes the inputs and
+outputs.
+
 Collected last (file name) so it also runs after every other GPU test has used
-the library; it passes alone too. Results are compared with fa_fwd_splitkv
-(caller workspace) on the same inputs, on two calls in a row, within the
-tolerances of the oracle comparisons.
+the library; it passes alone too. The static-scratch call runs the same
+kernels on the same inputs as fa_fwd_splitkv with a caller workspace, so the
+two results must agree bit for bit; that is checked on two calls in a row,
+and the device's free memory must not change across warm calls.
 """
 
 import pytest
 import torch
 
-from gpu_helpers import LSE_TOL, O_TOL
 from tiled_online_softmax_03_b200.inputs import Workload, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -27,13 +34,10 @@ def inputs(B, Hq, Hk, N, d, dtype, causal, seed):
     return w, tuple(x[n].to(dev) for n in ("q", "k", "v"))
 
 
-def assert_close(a, b, dtype):
+def assert_same(a, b):
     (oa, la), (ob, lb) = a, b
-    assert (oa.float() - ob.float()).abs().max().item() <= O_TOL[dtype]
-    fin = torch.isfinite(lb)
-    assert torch.equal(torch.isfinite(la), fin)
-    if fin.any():
-        assert (la[fin] - lb[fin]).abs().max().item() <= LSE_TOL
+    assert torch.equal(oa, ob), "O differs from the caller-workspace call"
+    assert torch.equal(la, lb), "LSE differs from the caller-workspace call"
 
 
 @pytest.mark.parametrize("B,Hq,Hk,N,d,dtype,causal,splits", [
@@ -43,19 +47,24 @@ def assert_close(a, b, dtype):
 ])
 def test_static_scratch_matches_caller_workspace_twice(B, Hq, Hk, N, d, dtype, causal, splits):
     from tiled_online_softmax_03_b200 import binding
-    w, (q, k, v) = inputs(B, Hq, Hk, N, d, dtype, causal, seed=N + splits)
+    _, (q, k, v) = inputs(B, Hq, Hk, N, d, dtype, causal, seed=N + splits)
     assert binding.splitkv_workspace_bytes(B, Hq, N, d, splits) <= binding.STATIC_SCRATCH_BYTES
     ref = binding.fa_fwd_splitkv(q, k, v, splits, causal=causal)
-    torch.cuda.synchronize()
     o = torch.empty_like(q)
     lse = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
+    # first call: may load the module and look up the scratch address
+    binding.fa_fwd_splitkv_static(q, k, v, splits, causal=causal, out=o, lse=lse)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
     for _ in range(2):  # two calls in a row on the same scratch
         o.fill_(7.0)
         lse.fill_(7.0)
         binding.fa_fwd_splitkv_static(q, k, v, splits, causal=causal, out=o, lse=lse)
         torch.cuda.synchronize()
         assert binding.device_status() == 0
-        assert_close((o, lse), ref, w.torch_dtype)
+        assert_same((o, lse), ref)
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, f"device free memory moved by {free0 - free1} bytes across warm calls"
 
 
 def test_static_scratch_rejects_problems_beyond_its_size():

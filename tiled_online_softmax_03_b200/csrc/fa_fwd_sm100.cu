@@ -1130,10 +1130,12 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 using AddressRangeFn = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
 
 struct DriverFns {
   EncodeTiledFn encode = nullptr;
   AddressRangeFn range = nullptr;
+  CtxGetCurrentFn ctx_current = nullptr;
   bool ok = false;
 };
 
@@ -1141,17 +1143,22 @@ const DriverFns& driver_fns() {
   static DriverFns fns;
   static std::once_flag once;
   std::call_once(once, [] {
-    cudaDriverEntryPointQueryResult q1, q2;
+    cudaDriverEntryPointQueryResult q1, q2, q3;
     void* f1 = nullptr;
     void* f2 = nullptr;
+    void* f3 = nullptr;
     if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f1, 12000, cudaEnableDefault,
                                          &q1) == cudaSuccess &&
         q1 == cudaDriverEntryPointSuccess &&
         cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &f2, 12000, cudaEnableDefault,
                                          &q2) == cudaSuccess &&
-        q2 == cudaDriverEntryPointSuccess) {
+        q2 == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f3, 12000, cudaEnableDefault,
+                                         &q3) == cudaSuccess &&
+        q3 == cudaDriverEntryPointSuccess) {
       fns.encode = reinterpret_cast<EncodeTiledFn>(f1);
       fns.range = reinterpret_cast<AddressRangeFn>(f2);
+      fns.ctx_current = reinterpret_cast<CtxGetCurrentFn>(f3);
       fns.ok = true;
     }
   });
@@ -1346,11 +1353,48 @@ int fa_unit_for(int cta, int it, int grid) { return fa::unit_for(cta, it, grid);
 
 }  // extern "C"
 
+// ============================================ split-KV with a static scratch
+// The scratch of fa_fwd_splitkv_static: a file-scope device array, so the
+// call allocates nothing. It exists once per device that loads this module
+// and is shared by every call on that device.
+static __device__ __align__(256) uint8_t g_fa_static_scratch[FA_STATIC_SCRATCH_BYTES];
+
+namespace {
+// Device address of g_fa_static_scratch per device, with the context it was
+// looked up in: a new primary context (after cudaDeviceReset) reloads the
+// module, so the address is looked up again when the current context differs.
+struct ScratchAddr {
+  CUcontext ctx = nullptr;
+  void* ptr = nullptr;
+};
+ScratchAddr g_scratch[64];
+
+int static_scratch(int dev, void** ptr) {
+  CUcontext ctx = nullptr;
+  if (driver_fns().ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+    return fail(FA_ERR_CUDA, "no current CUDA context");
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  ScratchAddr& a = g_scratch[dev];
+  if (a.ptr == nullptr || a.ctx != ctx) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_fa_static_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(FA_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s",
+                  cudaGetErrorString(e));
+    a.ctx = ctx;
+    a.ptr = p;
+  }
+  *ptr = a.ptr;
+  return FA_OK;
+}
+}  // namespace
+
 namespace {
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hk,
              int N, int d, float scale, int causal, const int32_t* key_pad_lens, int splits,
              void* workspace, size_t workspace_bytes, void* stream, int dtype,
-             const void* bias = nullptr, int bias_B = 0, int bias_H = 0) {
+             const void* bias = nullptr, int bias_B = 0, int bias_H = 0,
+             bool library_scratch = false) {
   g_err[0] = '\0';
   // ---- arguments that need no CUDA call
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr)
@@ -1436,9 +1480,21 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   prm.bias_H = bias_H > 0 ? bias_H : 1;
   if (splits > 1) {
     const size_t need = splitkv_bytes(heads_q, N, d, splits);
+    if (library_scratch) {
+      // fa_fwd_splitkv_static: the library's own scratch, after every other check
+      if (need > FA_STATIC_SCRATCH_BYTES)
+        return fail(FA_ERR_INVALID_ARG,
+                    "split-KV scratch of %zu bytes needed, the static scratch holds %zu; "
+                    "use fa_fwd_splitkv with a caller workspace",
+                    need, (size_t)FA_STATIC_SCRATCH_BYTES);
+      if ((rc = static_scratch(dev, &workspace)) != FA_OK) return rc;
+      workspace_bytes = FA_STATIC_SCRATCH_BYTES;
+    }
     if (workspace_bytes < need)
       return fail(FA_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", workspace_bytes, need);
-    if ((rc = check_range("workspace", workspace, need, 256)) != FA_OK) return rc;
+    // The library's own scratch is a module variable, not an allocation the
+    // range query knows; its size is checked above.
+    if (!library_scratch && (rc = check_range("workspace", workspace, need, 256)) != FA_OK) return rc;
     const uintptr_t wb = reinterpret_cast<uintptr_t>(workspace), we = wb + need;
     auto hits = [&](const void* x, size_t n) {
       const uintptr_t xb = reinterpret_cast<uintptr_t>(x);
@@ -1550,126 +1606,13 @@ int fa_selftest_wait_timeout(int ms) {
 
 }  // extern "C"
 
-// ============================================ split-KV with a static scratch
-// The scratch of fa_fwd_splitkv_static: a file-scope device array, so the
-// call allocates nothing. It exists once per device that loads this module
-// and is shared by every call on that device.
-static __device__ __align__(256) uint8_t g_fa_static_scratch[FA_STATIC_SCRATCH_BYTES];
-
-namespace {
-void* g_scratch_ptr[64] = {};  // device address of g_fa_static_scratch, per device
-
-// Device address of the scratch on the current device, looked up once.
-int static_scratch(int dev, void** ptr) {
-  std::lock_guard<std::mutex> lk(g_dev_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_fa_static_scratch);
-    if (e != cudaSuccess || p == nullptr)
-      return fail(FA_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s",
-                  cudaGetErrorString(e));
-    g_scratch_ptr[dev] = p;
-  }
-  *ptr = g_scratch_ptr[dev];
-  return FA_OK;
-}
-}  // namespace
 
 extern "C" int fa_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o,
                                      float* lse, int B, int Hq, int Hk, int N, int d, float scale,
                                      int causal, const int32_t* key_pad_lens, int num_splits,
                                      void* stream, int dtype) {
-  g_err[0] = '\0';
-  // ---- arguments that need no CUDA call (the rules of fa_fwd_splitkv)
-  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr)
-    return fail(FA_ERR_INVALID_ARG, "q, k, v and o must be non-NULL");
-  if (B < 1 || Hq < 1 || Hk < 1 || N < 1)
-    return fail(FA_ERR_INVALID_ARG, "B, Hq, Hk and N must be >= 1");
-  if (Hq % Hk != 0) return fail(FA_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hk (%d)", Hq, Hk);
-  if (d != 64 && d != 128)
-    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", d);
-  if (dtype != FA_FP16 && dtype != FA_BF16) return fail(FA_ERR_UNSUPPORTED, "unknown dtype %d", dtype);
-  if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "scale must be finite");
-  if (causal != 0 && causal != 1) return fail(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
-  if (num_splits < 1 || num_splits > 16)
-    return fail(FA_ERR_INVALID_ARG, "num_splits %d out of [1, 16]", num_splits);
-  const long long heads_q = (long long)B * Hq, heads_k = (long long)B * Hk;
-  if (heads_q > 0x7fffffffLL || N > (1 << 30))
-    return fail(FA_ERR_INVALID_ARG, "problem too large for 32-bit tile coordinates");
-  const int units = fa_num_units(B, Hq, Hk, N, causal);
-  if (units < 0) return FA_ERR_INVALID_ARG;
-  if ((long long)units * num_splits > 0x7fffffffLL)
-    return fail(FA_ERR_INVALID_ARG, "too many work units");
-  const size_t need = num_splits > 1 ? splitkv_bytes(heads_q, N, d, num_splits) : 0;
-  if (need > FA_STATIC_SCRATCH_BYTES)
-    return fail(FA_ERR_INVALID_ARG,
-                "split-KV scratch of %zu bytes needed, the static scratch holds %zu; "
-                "use fa_fwd_splitkv with a caller workspace",
-                need, (size_t)FA_STATIC_SCRATCH_BYTES);
-  // ---- device and buffers
-  if (!driver_fns().ok) return fail(FA_ERR_CUDA, "CUDA driver entry points unavailable");
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-    return fail(FA_ERR_CUDA, "no current CUDA device");
-  DeviceInfo& info = g_dev[dev];
-  {
-    std::lock_guard<std::mutex> lk(g_dev_mu);
-    if (!info.init) {
-      cudaDeviceProp prop;
-      if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess)
-        return fail(FA_ERR_CUDA, "cudaGetDeviceProperties failed");
-      info.sm100 = prop.major == 10 && prop.minor == 0;
-      info.sms = prop.multiProcessorCount;
-      info.init = true;
-    }
-  }
-  if (!info.sm100) return fail(FA_ERR_UNSUPPORTED, "device %d is not sm_100", dev);
-  void* scratch = nullptr;
-  int rc;
-  if (num_splits > 1 && (rc = static_scratch(dev, &scratch)) != FA_OK) return rc;
-  const size_t q_bytes = (size_t)heads_q * N * d * 2, kv_bytes = (size_t)heads_k * N * d * 2;
-  if ((rc = check_range("q", q, q_bytes, 16)) != FA_OK) return rc;
-  if ((rc = check_range("k", k, kv_bytes, 16)) != FA_OK) return rc;
-  if ((rc = check_range("v", v, kv_bytes, 16)) != FA_OK) return rc;
-  if ((rc = check_range("o", o, q_bytes, 16)) != FA_OK) return rc;
-  if (lse != nullptr && (rc = check_range("lse", lse, (size_t)heads_q * N * 4, 4)) != FA_OK) return rc;
-  if (key_pad_lens != nullptr &&
-      (rc = check_range("key_pad_lens", key_pad_lens, (size_t)B * 4, 4)) != FA_OK)
-    return rc;
-  const uintptr_t ob = reinterpret_cast<uintptr_t>(o), oe = ob + q_bytes;
-  auto overlaps = [&](const void* x, size_t n) {
-    const uintptr_t xb = reinterpret_cast<uintptr_t>(x);
-    return xb < oe && ob < xb + n;
-  };
-  if (overlaps(q, q_bytes) || overlaps(k, kv_bytes) || overlaps(v, kv_bytes) ||
-      (lse != nullptr && overlaps(lse, (size_t)heads_q * N * 4)))
-    return fail(FA_ERR_INVALID_ARG, "o overlaps an input or lse");
-
-  fa::Params prm;
-  prm.key_pad_lens = key_pad_lens;
-  prm.lse = lse;
-  prm.o_part = nullptr;
-  prm.lse_part = nullptr;
-  prm.o_scale = 1.f;
-  prm.bias_bmul = 0;
-  prm.bias_hmul = 0;
-  prm.bias_H = 1;
-  if (num_splits > 1) {
-    const size_t rows = (size_t)heads_q * N * num_splits;
-    prm.o_part = reinterpret_cast<float*>(scratch);
-    prm.lse_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(scratch) +
-                                            (rows * d * 4 + 255) / 256 * 256);
-  }
-  prm.s = fa::make_shape(B, Hq, Hk, N, causal, num_splits);
-  prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
-  prm.timeout_ns = g_timeout_ns;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const bool bf16 = dtype == FA_BF16;
-  if (d == 128)
-    return bf16 ? launch<128, true>(q, k, v, o, prm, st, info, 0, lse)
-                : launch<128, false>(q, k, v, o, prm, st, info, 1, lse);
-  return bf16 ? launch<64, true>(q, k, v, o, prm, st, info, 2, lse)
-              : launch<64, false>(q, k, v, o, prm, st, info, 3, lse);
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hk, N, d, scale, causal, key_pad_lens, num_splits,
+                  nullptr, 0, stream, dtype, nullptr, 0, 0, /*library_scratch=*/true);
 }
 
 // ================================================================ backward
