@@ -249,6 +249,55 @@ int fa_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o, 
                           const int32_t* key_pad_lens, int num_splits, void* stream,
                           int dtype);
 
+/*
+ * fa_fwd_host — fa_fwd on inputs and outputs in HOST memory, with the PCIe
+ * copies overlapped with the attention. The pages' user-level call takes whole
+ * Q, K, V tensors and returns O (NPU page "FlashAttention 在昇腾 NPU 上是怎么省
+ * 显存的？我花了两天把它搞明白了", usage section: flash_attention(q, k, v,
+ * block_size, causal)); this is that call for tensors that live on the host.
+ *
+ *   q, k, v        PINNED host memory (cudaMallocHost, cudaHostAlloc or
+ *                  cudaHostRegister), layouts as for fa_fwd; read by
+ *                  asynchronous copies after the call returns.
+ *   o              pinned host [B, Hq, N, d], written asynchronously.
+ *   lse            pinned host [B, Hq, N] float32, or NULL (then lse_dev NULL).
+ *   key_pad_lens   pinned host int32 [B] or NULL (no padding).
+ *   q_dev .. lens_dev  device buffers of the same sizes (lens_dev [B] int32,
+ *                  only with key_pad_lens), owned by the caller; they hold the
+ *                  staged inputs and outputs and must not overlap.
+ *   num_chunks     0 (library's choice: about 16 MB of inputs per chunk, at
+ *                  most 16) or 1..64 wanted chunks: num_chunks runs of whole
+ *                  batches when B >= num_chunks, else every batch cut into
+ *                  min(Hk, ceil(num_chunks / B)) runs of K/V heads (with their
+ *                  query heads); fa_host_chunk_plan lists them.
+ *   stream         the caller's stream; other arguments as for fa_fwd.
+ *
+ * Per chunk: the copy in (q, k, v slices) on a library copy stream, fa_fwd on
+ * the chunk's slices on `stream`, the copy out (o, lse slices) on a second
+ * library copy stream, ordered by events, so copies in, kernels and copies
+ * out of different chunks overlap. The copy streams wait for the work already
+ * on `stream`, and `stream` waits for every copy before returning: once
+ * `stream` has been synchronised (or waited on), o and lse hold the result
+ * and the host inputs may be rewritten. Not before: until then the host
+ * inputs must not be written and the outputs not read.
+ *
+ * Allocates no device memory. The first call on a device creates the two
+ * copy streams (kept for the life of the process); each call creates and
+ * releases four events. Errors: FA_ERR_INVALID_ARG for pageable host memory,
+ * bad sizes, overlapping device buffers; otherwise as fa_fwd. On an error
+ * after copies were enqueued, `stream` is still ordered after them.
+ */
+int fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                int Hk, int N, int d, float scale, int causal, const int32_t* key_pad_lens,
+                void* q_dev, void* k_dev, void* v_dev, void* o_dev, float* lse_dev,
+                int32_t* lens_dev, int num_chunks, void* stream, int dtype);
+
+/* The chunks fa_fwd_host uses for a shape and num_chunks (0: its default):
+ * writes {b0, b1, hk0, hk1} per chunk to out[4 * i ..], at most max_chunks
+ * chunks, and returns their count (< 0 on bad arguments). Host only. */
+int fa_host_chunk_plan(int B, int Hq, int Hk, int N, int d, int num_chunks, int32_t* out,
+                       int max_chunks);
+
 /* Message for the last error returned to the calling thread ("" if none).
  * The string is owned by the library (thread-local storage). */
 const char* fa_last_error_string(void);

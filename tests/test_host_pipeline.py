@@ -1,8 +1,9 @@
-"""fa_fwd_from_host: the forward on pinned host buffers, pipelined batch by
-batch (copy in of b + 1, attention of b, copy out of b − 1 on three streams).
-Each batch runs the same kernel on its slices, so the result must equal the
-device-buffer fa_fwd bit for bit; the oracle comparison of fa_fwd itself is in
-test_parity.py.
+"""fa_fwd_host (binding: fa_fwd_from_host): the forward on pinned host
+buffers, pipelined chunk by chunk (copy in of chunk c + 1, attention of chunk
+c, copy out of chunk c − 1 on three streams). Each chunk runs the same kernel
+on its slices (whole batches, or runs of K/V heads of one batch), so the
+result must equal the device-buffer fa_fwd bit for bit; the oracle comparison
+of fa_fwd itself is in test_parity.py.
 """
 
 import pytest
@@ -47,20 +48,43 @@ def test_equals_device_call_bitwise(B, Hq, Hk, N, d, dtype, causal, lens):
     assert torch.equal(o, o_ref.cpu()) and torch.equal(lse, l_ref.cpu())
 
 
-@pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 6, 31, 32, 33])
-@pytest.mark.parametrize("chunks", [None, 1, 2, 3, 100])
-def test_chunk_ranges_partition_the_batch(B, chunks):
-    from tiled_online_softmax_03_b200.binding import chunk_ranges
-    r = chunk_ranges(B, chunks)
-    assert r[0][0] == 0 and r[-1][1] == B
-    assert all(a1 == b0 for (_, a1), (b0, _) in zip(r, r[1:]))
-    sizes = [b1 - b0 for b0, b1 in r]
-    assert min(sizes) >= 1 and max(sizes) - min(sizes) <= 1
-    assert len(r) == (min(B, 4) if chunks is None else min(chunks, B))
+@pytest.mark.parametrize("B,Hq,Hk", [(1, 32, 8), (1, 32, 32), (1, 1, 1), (2, 4, 2), (3, 8, 8),
+                                      (4, 32, 8), (4, 32, 1), (32, 16, 16), (33, 2, 1)])
+@pytest.mark.parametrize("chunks", [0, 1, 2, 3, 5, 16, 64])
+def test_chunk_plan_covers_every_head_once(B, Hq, Hk, chunks):
+    """Every (b, K/V head) lands in exactly one chunk; a chunk is one
+    contiguous slice (whole batches, or a run of K/V heads of one batch)."""
+    from tiled_online_softmax_03_b200.binding import host_chunk_plan
+    N, d = 4096, 128
+    plan = host_chunk_plan(B, Hq, Hk, N, d, chunks)
+    seen = []
+    for b0, b1, h0, h1 in plan:
+        assert 0 <= b0 < b1 <= B and 0 <= h0 < h1 <= Hk
+        if b1 - b0 > 1:
+            assert (h0, h1) == (0, Hk), "a multi-batch chunk must hold every head"
+        seen += [(b, h) for b in range(b0, b1) for h in range(h0, h1)]
+    assert seen == [(b, h) for b in range(B) for h in range(Hk)]  # in order, once each
+    if chunks:
+        if B >= chunks:
+            assert len(plan) == chunks
+        else:
+            assert len(plan) == B * min(Hk, -(-chunks // B))
+    else:  # default: about 16 MB of inputs per chunk, at most 16 chunks
+        mb = 2 * B * N * d * (Hq + 2 * Hk) / 2 ** 20
+        want = max(1, min(16, int(mb // 16)))
+        assert len(plan) == (want if B >= want else B * min(Hk, -(-want // B)))
+
+
+def test_chunk_plan_rejects_bad_arguments():
+    from tiled_online_softmax_03_b200 import binding
+    for args in [(0, 1, 1, 8, 64, 0), (1, 3, 2, 8, 64, 0), (1, 1, 1, 8, 64, -1),
+                 (1, 1, 1, 8, 64, 65)]:
+        with pytest.raises(binding.FaError):
+            binding.host_chunk_plan(*args)
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("chunks", [None, 1, 3, 6])
+@pytest.mark.parametrize("chunks", [None, 1, 3, 6, 12])
 def test_multi_batch_chunks_equal_device_call(chunks):
     from tiled_online_softmax_03_b200 import binding
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
@@ -97,6 +121,75 @@ def test_reused_buffers_across_calls():
     for x, o, lse in results:
         o_ref, l_ref = binding.fa_fwd(x["q"].to(dev), x["k"].to(dev), x["v"].to(dev), causal=True)
         assert torch.equal(o, o_ref.cpu()) and torch.equal(lse, l_ref.cpu())
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("B,Hq,Hk,chunks", [(1, 8, 2, 2), (1, 8, 8, 5), (2, 8, 4, 4), (1, 4, 1, 3)])
+def test_head_chunks_equal_device_call(B, Hq, Hk, chunks):
+    """Chunks that cut a batch into runs of K/V heads (B below the chunk count)."""
+    from tiled_online_softmax_03_b200 import binding
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    w, x, L = _host_inputs(B, Hq, Hk, 700, 128, "bf16", True, [650, 333][:B], seed=3 + B + Hk)
+    dev = torch.device("cuda:0")
+    o_ref, l_ref = binding.fa_fwd(x["q"].to(dev), x["k"].to(dev), x["v"].to(dev), causal=True,
+                                  key_pad_lens=L.to(dev))
+    hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
+    assert len(binding.host_chunk_plan(B, Hq, Hk, 700, 128, chunks)) > B
+    o, lse = binding.fa_fwd_from_host(hq, hk, hv, causal=True, key_pad_lens=L.pin_memory(),
+                                      chunks=chunks)
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    assert torch.equal(o, o_ref.cpu()) and torch.equal(lse, l_ref.cpu())
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("as_handle", [False, True])
+def test_side_stream_with_owned_buffers(as_handle):
+    """Two calls on a side stream (a torch stream, or its raw handle) with the
+    device buffers allocated by the call, and allocations on the current
+    stream in between: both results equal fa_fwd bit for bit."""
+    from tiled_online_softmax_03_b200 import binding
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    dev = torch.device("cuda:0")
+    side = torch.cuda.Stream(dev)
+    B, Hq, Hk, N, d = 2, 8, 2, 1024, 128
+    results = []
+    for seed in (21, 22):
+        w, x, _ = _host_inputs(B, Hq, Hk, N, d, "bf16", True, seed=seed)
+        hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
+        o, lse = binding.fa_fwd_from_host(hq, hk, hv, causal=True, device=dev,
+                                          stream=side.cuda_stream if as_handle else side)
+        junk = [torch.full((1 << 20,), 3.0, device=dev) for _ in range(8)]  # reuse pressure
+        del junk
+        results.append((x, o, lse))
+    side.synchronize()
+    assert binding.device_status() == 0
+    for x, o, lse in results:
+        o_ref, l_ref = binding.fa_fwd(x["q"].to(dev), x["k"].to(dev), x["v"].to(dev), causal=True)
+        assert torch.equal(o, o_ref.cpu()) and torch.equal(lse, l_ref.cpu())
+
+
+@pytest.mark.gpu
+def test_stream_on_another_device_or_pageable_memory_is_refused():
+    from tiled_online_softmax_03_b200 import binding
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    B, Hq, Hk, N, d = 1, 2, 1, 128, 64
+    w, x, _ = _host_inputs(B, Hq, Hk, N, d, "bf16", False, seed=2)
+    hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
+    if torch.cuda.device_count() > 1:
+        with pytest.raises(binding.FaError, match="stream"):
+            binding.fa_fwd_from_host(hq, hk, hv, device=torch.device("cuda:0"),
+                                     stream=torch.cuda.Stream(torch.device("cuda:1")))
+    # the C call itself refuses pageable host memory
+    dev = torch.device("cuda:0")
+    bufs = [torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (hq, hk, hv, hq)]
+    lse_d = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    out = torch.empty(hq.shape, dtype=hq.dtype)  # not pinned
+    rc = binding.lib.fa_fwd_host(hq.data_ptr(), hk.data_ptr(), hv.data_ptr(), out.data_ptr(), None,
+                                 B, Hq, Hk, N, d, 0.125, 0, None, bufs[0].data_ptr(),
+                                 bufs[1].data_ptr(), bufs[2].data_ptr(), bufs[3].data_ptr(), None,
+                                 None, 0, None, binding.FA_BF16)
+    assert rc == binding.FA_ERR_INVALID_ARG and "pinned" in binding.last_error()
 
 
 class _FakeDev:

@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["FaError", "fa_fwd", "fa_bwd", "fa_fwd_fp8", "fa_fwd_bias", "fa_fwd_splitkv", "splitkv_workspace_bytes", "load_library", "lib", "FA_OK", "FA_ERR_INVALID_ARG",
+__all__ = ["FaError", "fa_fwd", "fa_fwd_from_host", "host_chunk_plan", "fa_bwd", "fa_fwd_fp8", "fa_fwd_bias", "fa_fwd_splitkv", "splitkv_workspace_bytes", "load_library", "lib", "FA_OK", "FA_ERR_INVALID_ARG",
            "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT"]
 
 FA_OK = 0
@@ -65,6 +65,11 @@ def load_library(path=LIB_PATH):
                                         c_int, c_int, c_int, c_int, c_float, c_int, c_void_p,
                                         c_int, c_void_p, c_int]
     L.fa_fwd_splitkv_static.restype = c_int
+    L.fa_fwd_host.argtypes = [c_void_p] * 5 + [c_int] * 5 + [c_float, c_int, c_void_p] + \
+        [c_void_p] * 6 + [c_int, c_void_p, c_int]
+    L.fa_fwd_host.restype = c_int
+    L.fa_host_chunk_plan.argtypes = [c_int] * 6 + [ctypes.POINTER(ctypes.c_int32), c_int]
+    L.fa_host_chunk_plan.restype = c_int
     L.fa_splitkv_workspace_bytes.argtypes = [c_int] * 5
     L.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
     L.fa_unit_kv_range.argtypes = [c_int] * 8 + [ctypes.POINTER(ctypes.c_int32)]
@@ -148,37 +153,43 @@ def fa_fwd(q, k, v, causal=False, scale=None, key_pad_lens=None, out=None, lse=N
     return (out, lse) if return_lse else out
 
 
-_IO_STREAMS = {}
-
-
-def _io_streams(device):
-    """Two streams per device for the copies in and out of fa_fwd_from_host."""
-    key = device.index
-    if key not in _IO_STREAMS:
-        _IO_STREAMS[key] = (torch.cuda.Stream(device), torch.cuda.Stream(device))
-    return _IO_STREAMS[key]
+def _stream_handle(stream, device):
+    """(raw cudaStream_t handle, torch stream object or None) for ``stream``: a
+    torch.cuda.Stream, a raw handle (int), or None for the device's current
+    stream. A torch stream on another device is refused."""
+    if stream is None:
+        st = torch.cuda.current_stream(device)
+        return st.cuda_stream, st
+    if isinstance(stream, torch.cuda.Stream):
+        if stream.device != device:
+            raise FaError(FA_ERR_INVALID_ARG, f"stream is on {stream.device}, not {device}")
+        return stream.cuda_stream, stream
+    if isinstance(stream, int):
+        return stream, torch.cuda.ExternalStream(stream, device=device)
+    raise FaError(FA_ERR_INVALID_ARG, "stream must be a torch.cuda.Stream, a raw handle or None")
 
 
 def fa_fwd_from_host(q, k, v, causal=False, scale=None, key_pad_lens=None, out=None, lse=None,
                      device_buffers=None, device=None, stream=None, chunks=None):
-    """fa_fwd on page-locked HOST tensors, pipelined chunk by chunk of the batch.
+    """``fa_fwd_host`` of the C ABI: the forward on page-locked HOST tensors.
 
     q [B,Hq,N,d], k and v [B,Hk,N,d] (and key_pad_lens, int32 [B], if given)
     are contiguous pinned CPU tensors; ``out`` [B,Hq,N,d] and ``lse``
     [B,Hq,N] float32, pinned CPU tensors, receive the result (allocated pinned
-    when None). The device copies live in ``device_buffers``, a dict of CUDA
-    tensors 'q', 'k', 'v', 'o', 'lse' of the same shapes and, with padding,
-    'lens' [B] int32; they are allocated on ``device`` (default: the current
-    CUDA device) when None. The batch is cut into ``chunks`` near-equal runs
-    of consecutive batches (default min(B, 4): large enough copies, and
-    launches that still fill the GPU); for each chunk c the copy in of chunk
-    c + 1, the attention of chunk c (one fa_fwd call of the C ABI on the
-    chunk's slices) and the copy out of chunk c − 1 run on three streams, so
-    the two PCIe directions and the kernel overlap. The kernels go on ``stream`` (a
-    torch.cuda.Stream; default the current stream), which on return is ordered
-    after every copy: synchronising it makes ``out`` and ``lse`` valid.
-    Consecutive calls on one stream do not overlap each other. Caller-given
-    device buffers must stay alive until then. Returns (out, lse).
+    when None). The staged device copies live in ``device_buffers``, a dict of
+    CUDA tensors 'q', 'k', 'v', 'o', 'lse' of the same shapes and, with
+    padding, 'lens' [B] int32; they are allocated on ``device`` (default: the
+    current CUDA device) when None. The library cuts the work into ``chunks``
+    (None: its default, about 16 MB of inputs each) and overlaps, chunk by
+    chunk, the copy in, the attention and the copy out.
+
+    ``stream`` is a torch.cuda.Stream or a raw cudaStream_t handle on
+    ``device`` (default: its current stream). The call returns once the work
+    is enqueued. Only after ``stream`` has been synchronised (or waited on)
+    do ``out`` and ``lse`` hold the result, and only then may q, k, v and
+    key_pad_lens be written again: asynchronous copies read them until then.
+    Caller-given device buffers must also stay alive until then. Returns
+    (out, lse).
     """
     for name, t in (("q", q), ("k", k), ("v", v)):
         if t.is_cuda or not t.is_contiguous() or t.dim() != 4 or not t.is_pinned():
@@ -212,13 +223,14 @@ def fa_fwd_from_host(q, k, v, causal=False, scale=None, key_pad_lens=None, out=N
         device = torch.device("cuda", torch.cuda.current_device())
     owned = device_buffers is None
     if owned:
-        device_buffers = {"q": torch.empty(q.shape, dtype=q.dtype, device=device),
-                          "k": torch.empty(k.shape, dtype=q.dtype, device=device),
-                          "v": torch.empty(v.shape, dtype=q.dtype, device=device),
-                          "o": torch.empty(q.shape, dtype=q.dtype, device=device),
-                          "lse": torch.empty((B, Hq, N), dtype=torch.float32, device=device),
-                          "lens": (torch.empty(B, dtype=torch.int32, device=device)
-                                   if key_pad_lens is not None else None)}
+        with torch.cuda.device(device):
+            device_buffers = {"q": torch.empty(q.shape, dtype=q.dtype, device=device),
+                              "k": torch.empty(k.shape, dtype=q.dtype, device=device),
+                              "v": torch.empty(v.shape, dtype=q.dtype, device=device),
+                              "o": torch.empty(q.shape, dtype=q.dtype, device=device),
+                              "lse": torch.empty((B, Hq, N), dtype=torch.float32, device=device),
+                              "lens": (torch.empty(B, dtype=torch.int32, device=device)
+                                       if key_pad_lens is not None else None)}
     want = {"q": (tuple(q.shape), q.dtype), "k": (tuple(k.shape), q.dtype), "v": (tuple(v.shape), q.dtype),
             "o": (tuple(q.shape), q.dtype), "lse": ((B, Hq, N), torch.float32)}
     if key_pad_lens is not None:
@@ -231,48 +243,31 @@ def fa_fwd_from_host(q, k, v, causal=False, scale=None, key_pad_lens=None, out=N
                           f"device_buffers['{n}'] must be a contiguous {dt} tensor {list(shape)} on {device}")
     qd, kd, vd, od, ld = (device_buffers[n] for n in ("q", "k", "v", "o", "lse"))
     lens_d = device_buffers["lens"] if key_pad_lens is not None else None
-    cs = torch.cuda.current_stream(device) if stream is None else stream
-    s_in, s_out = _io_streams(device)
+    handle, st = _stream_handle(stream, device)
     if owned:
+        # the library's copy streams finish before `stream` does: tying the
+        # buffers to `stream` keeps them alive until every copy has run
         for t in (qd, kd, vd, od, ld) + ((lens_d,) if lens_d is not None else ()):
-            t.record_stream(s_in)
-            t.record_stream(s_out)
-    # earlier work on the stream, the previous call's copies out included,
-    # comes first: the device buffers are reused
-    cs.wait_stream(s_out)
-    s_in.wait_stream(cs)
-    s_out.wait_stream(cs)
-    if lens_d is not None:
-        with torch.cuda.stream(s_in):
-            lens_d.copy_(key_pad_lens, non_blocking=True)
-    for b0, b1 in chunk_ranges(B, chunks):
-        with torch.cuda.stream(s_in):
-            qd[b0:b1].copy_(q[b0:b1], non_blocking=True)
-            kd[b0:b1].copy_(k[b0:b1], non_blocking=True)
-            vd[b0:b1].copy_(v[b0:b1], non_blocking=True)
-        cs.wait_event(s_in.record_event())
-        fa_fwd(qd[b0:b1], kd[b0:b1], vd[b0:b1], causal=causal, scale=scale,
-               key_pad_lens=lens_d[b0:b1] if lens_d is not None else None,
-               out=od[b0:b1], lse=ld[b0:b1], stream=cs.cuda_stream)
-        s_out.wait_event(cs.record_event())
-        with torch.cuda.stream(s_out):
-            out[b0:b1].copy_(od[b0:b1], non_blocking=True)
-            lse[b0:b1].copy_(ld[b0:b1], non_blocking=True)
-    cs.wait_stream(s_out)
+            t.record_stream(st)
+    if scale is None:
+        scale = float(d) ** -0.5
+    with torch.cuda.device(device):
+        check(lib.fa_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                              lse.data_ptr(), B, Hq, Hk, N, d, float(scale), 1 if causal else 0,
+                              key_pad_lens.data_ptr() if key_pad_lens is not None else None,
+                              qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
+                              ld.data_ptr(), lens_d.data_ptr() if lens_d is not None else None,
+                              0 if chunks is None else int(chunks), handle, _DTYPES[q.dtype]))
     return out, lse
 
 
-def chunk_ranges(B, chunks=None):
-    """[b0, b1) runs of consecutive batches: ``chunks`` (default min(B, 4))
-    near-equal parts, the first B % chunks one batch longer."""
-    n = min(B, 4) if chunks is None else max(1, min(int(chunks), B))
-    base, extra = divmod(B, n)
-    out, b0 = [], 0
-    for i in range(n):
-        b1 = b0 + base + (1 if i < extra else 0)
-        out.append((b0, b1))
-        b0 = b1
-    return out
+def host_chunk_plan(B, Hq, Hk, N, d, chunks=None):
+    """[(b0, b1, hk0, hk1)] chunks fa_fwd_host uses (chunks None: its default)."""
+    out = (ctypes.c_int32 * (4 * 64))()
+    n = lib.fa_host_chunk_plan(B, Hq, Hk, N, d, 0 if chunks is None else int(chunks), out, 64)
+    if n < 0:
+        check(n)
+    return [tuple(out[4 * i:4 * i + 4]) for i in range(n)]
 
 
 def fa_fwd_bias(q, k, v, bias, causal=False, scale=None, key_pad_lens=None, out=None, lse=None,

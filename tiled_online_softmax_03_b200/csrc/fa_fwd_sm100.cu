@@ -1899,3 +1899,5 @@ extern "C" int fa_fwd_fp8(const void* q, const void* k, const void* v, float q_d
   prm.timeout_ns = g_timeout_ns;
   return launch<128, true, 2>(q, k, vt, o, prm, st, info, 8, lse);
 }
+
+#include "fa_host_pipeline.cuh"
