@@ -124,7 +124,7 @@ def test_reused_buffers_across_calls():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("B,Hq,Hk,chunks", [(1, 8, 2, 2), (1, 8, 8, 5), (2, 8, 4, 4), (1, 4, 1, 3)])
+@pytest.mark.parametrize("B,Hq,Hk,chunks", [(1, 8, 2, 2), (1, 8, 8, 5), (2, 8, 4, 4), (1, 4, 4, 3)])
 def test_head_chunks_equal_device_call(B, Hq, Hk, chunks):
     """Chunks that cut a batch into runs of K/V heads (B below the chunk count)."""
     from tiled_online_softmax_03_b200 import binding

@@ -54,29 +54,48 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: keep a stale max until
 constexpr int SW128_BOX_BYTES = BM * 128;  // one 128-row box of 64 16-bit columns
 constexpr int OST_BYTES = 32 * 32 * 2;     // one 32-row × 32-column output staging box
 
-// TMEM columns: S/P for tile 0 and 1, then O for tile 0 and 1.
+// TMEM columns: S/P for tile 0 and 1, then O. At d = 128 the four regions
+// fill the 512 columns.
+//
+// Short-sequence configuration (d = 64): units hold only a few K/V tiles, so
+// the unit boundary matters as much as the steady state. There the Q tiles
+// and O are double-buffered (a unit's Q tiles load during the previous unit;
+// its first P·V does not wait for the previous unit's epilogue to read O
+// out: TMEM has 128 spare columns), units are decoded once into a ring of
+// records in shared memory, and the MMA warp issues the next unit's first S
+// right behind each tile's last P·V.
 __device__ constexpr uint32_t S_COL[2] = {0, 128};
 template <int D>
 struct TmemO {
-  __host__ __device__ static constexpr uint32_t col(int t) { return 256 + t * D; }
+  static constexpr bool SHORT = D == 64;
+  static constexpr int BUFS = SHORT ? 2 : 1;  // O buffers per tile
+  // final-statistics buffers per tile: a unit's softmax may finish while the
+  // epilogues of the BUFS units before it are still pending
+  static constexpr int NSTATS = SHORT ? 4 : 2;
+  __host__ __device__ static constexpr uint32_t col(int t, int buf) { return 256 + (t + 2 * buf) * D; }
 };
+
+constexpr int UNIT_RING = 4;
+constexpr int OFF_URING = 576;  // [UNIT_RING] × 64 bytes, after the barriers
 
 // Barrier slots.
 enum {
-  BAR_QFULL = 0,    // [2] TMA -> MMA: Q tile loaded
-  BAR_QEMPTY = 2,   // [2] MMA -> TMA: the unit's last QK no longer needs the Q tile
-  BAR_SFULL = 4,    // [2] MMA -> softmax: S tile ready in TMEM
-  BAR_PFULL = 6,    // [2] softmax -> MMA: P written to TMEM
-  BAR_AFULL = 8,    // [2] softmax -> correction: rescale factors in smem
-  BAR_OCORR = 10,   // [2] correction -> MMA: O rescaled
-  BAR_PVDONE = 12,  // [2] MMA -> epilogue: last P·V of the unit done
-  BAR_OFREE = 14,   // [2] epilogue -> MMA: O read out of TMEM
-  BAR_STATS = 16,   // [2 tiles][2 buffers] softmax -> epilogue: final m, l in smem
-  BAR_DRAIN = 20,   // MMA drain on the abort path
-  BAR_PHALF = 21,   // [2] softmax -> MMA: P of the first 64 keys written to TMEM
-  BAR_BFULL = 23,   // [2] TMA -> softmax: bias tile loaded (bias mode)
-  BAR_BEMPTY = 25,  // [2] softmax -> TMA: bias tile read
-  BAR_KV = 27       // [STAGES] full, then [STAGES] empty
+  BAR_QFULL = 0,    // [2 tiles][2 Q buffers] TMA -> MMA: Q tile loaded
+  BAR_QEMPTY = 4,   // [2 tiles][2 Q buffers] MMA -> TMA: the unit's last QK no longer needs it
+  BAR_SFULL = 8,    // [2] MMA -> softmax: S tile ready in TMEM
+  BAR_PFULL = 10,   // [2] softmax -> MMA: P written to TMEM
+  BAR_AFULL = 12,   // [2] softmax -> correction: rescale factors in smem
+  BAR_OCORR = 14,   // [2] correction -> MMA: O rescaled
+  BAR_PVDONE = 16,  // [2 tiles][2 O buffers] MMA -> epilogue: last P·V of the unit done
+  BAR_OFREE = 20,   // [2 tiles][2 O buffers] epilogue -> MMA: O read out of TMEM
+  BAR_STATS = 24,   // [2 tiles][4 buffers] softmax -> epilogue: final m, l in smem
+  BAR_DRAIN = 32,   // MMA drain on the abort path
+  BAR_PHALF = 33,   // [2] softmax -> MMA: P of the first 64 keys written to TMEM
+  BAR_BFULL = 35,   // [2] TMA -> softmax: bias tile loaded (bias mode)
+  BAR_BEMPTY = 37,  // [2] softmax -> TMA: bias tile read
+  BAR_UFULL = 39,   // [UNIT_RING] producer -> every role: unit record written (d = 64)
+  BAR_UEMPTY = 43,  // [UNIT_RING] every role -> producer: unit record read (d = 64)
+  BAR_KV = 47       // [STAGES] full, then [STAGES] empty
 };
 
 // Shared memory: barriers and flags first, then 1 KB-aligned tiles. With an
@@ -87,6 +106,8 @@ template <int D, int MODE = 0>
 struct Layout {
   static constexpr bool BIAS = MODE == 1, FP8 = MODE == 2;
   static constexpr int ELEM = FP8 ? 1 : 2;  // bytes per Q, K, V element
+  static constexpr bool RING = TmemO<D>::SHORT;  // unit ring, early next-unit S
+  static constexpr int QBUF = TmemO<D>::SHORT ? 2 : 1;
   static constexpr int Q_BYTES = BM * D * ELEM;
   static constexpr int KV_BYTES = BN * D * ELEM;
   static constexpr int STAGES = BIAS ? ((D == 128) ? 2 : 4) : ((D == 128 && !FP8) ? 4 : 8);
@@ -95,14 +116,14 @@ struct Layout {
   static constexpr int OFF_BAR = 0;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;     // tmem base, abort flag
   static constexpr int OFF_Q = 1024;
-  static constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_KV = OFF_Q + 2 * QBUF * Q_BYTES;  // Q: [QBUF][2 tiles]
   static constexpr int OFF_BIAS = OFF_KV + STAGES * KV_BYTES;  // [2 tiles] bias mode only
   static constexpr int OFF_OST = OFF_BIAS + 2 * BIAS_BYTES;
   static constexpr int OFF_ALPHA = OFF_OST + 8 * OST_BYTES;   // [2 tiles][128] float
-  static constexpr int OFF_STATS = OFF_ALPHA + 2 * BM * 4;    // [2 buf][2 tiles][128] float4
-  static constexpr int BYTES = OFF_STATS + 2 * 2 * BM * 16;
+  static constexpr int OFF_STATS = OFF_ALPHA + 2 * BM * 4;    // [NSTATS buf][2 tiles][128] float4
+  static constexpr int BYTES = OFF_STATS + TmemO<D>::NSTATS * 2 * BM * 16;
   static constexpr int ALLOC = BYTES + 1024;                  // base is rounded up to 1 KB
-  static_assert(OFF_MISC + 16 <= OFF_Q, "barrier area");
+  static_assert(OFF_MISC + 16 <= OFF_URING && OFF_URING + UNIT_RING * 64 <= OFF_Q, "barrier area");
   static_assert(OFF_KV % 1024 == 0 && OFF_BIAS % 1024 == 0 && OFF_OST % 1024 == 0,
                 "tile alignment");
   static_assert(ALLOC <= 232448, "shared memory budget");
@@ -200,6 +221,7 @@ __device__ __forceinline__ int key_len_of(const Params& p, int b) {
   return l < 0 ? 0 : (l > p.s.N ? p.s.N : l);
 }
 
+// Unit `it` of this CTA (serpentine order), decoded; false past the last one.
 __device__ __forceinline__ bool next_unit(const Params& p, int it, Unit& U) {
   const int u = unit_for(blockIdx.x, it, gridDim.x);
   if (u >= p.s.num_units) return false;
@@ -208,36 +230,103 @@ __device__ __forceinline__ bool next_unit(const Params& p, int it, Unit& U) {
   return true;
 }
 
+// Unit records: 16 ints, {valid, b, hk, split, hq0, hq1, mb0, mb1, present0,
+// present1, key_len, j0, n0, n1, nmax, -}; valid = 0 ends the walk.
+__device__ __forceinline__ void write_unit(uint8_t* smem, int slot, const Unit& U, int valid) {
+  int4* d = reinterpret_cast<int4*>(smem + OFF_URING + slot * 64);
+  d[0] = make_int4(valid, U.b, U.hk, U.split);
+  d[1] = make_int4(U.hq[0], U.hq[1], U.mb[0], U.mb[1]);
+  d[2] = make_int4(U.present[0], U.present[1], U.key_len, U.j0);
+  d[3] = make_int4(U.n[0], U.n[1], U.nmax, 0);
+}
+__device__ __forceinline__ int read_unit(const uint8_t* smem, int slot, Unit& U) {
+  const int4* r = reinterpret_cast<const int4*>(smem + OFF_URING + slot * 64);
+  const int4 a = r[0], b = r[1], c = r[2], d = r[3];
+  U.b = a.y; U.hk = a.z; U.split = a.w;
+  U.hq[0] = b.x; U.hq[1] = b.y; U.mb[0] = b.z; U.mb[1] = b.w;
+  U.present[0] = c.x; U.present[1] = c.y; U.key_len = c.z; U.j0 = c.w;
+  U.n[0] = d.x; U.n[1] = d.y; U.nmax = d.z;
+  return a.x;
+}
+// Record `it` for a whole warp: wait until it is written, copy it, release
+// the slot (one arrival per warp). 1: a unit, 0: no more units, -1: the wait
+// gave up.
+__device__ __forceinline__ int take_unit_warp(const uint8_t* smem, uint32_t sbase, int it,
+                                              const Ctl& c, Unit& U) {
+  const int slot = it & (UNIT_RING - 1);
+  if (!wait_bar_warp(bar_addr(sbase, BAR_UFULL + slot), (it / UNIT_RING) & 1, c)) return -1;
+  const int valid = read_unit(smem, slot, U);
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar_addr(sbase, BAR_UEMPTY + slot));
+  return valid;
+}
+// Unit `it` for a role: from the unit ring (RING), else decoded here.
+template <bool RING>
+__device__ __forceinline__ int get_unit_warp(const Params& p, const uint8_t* smem, uint32_t sbase,
+                                             int it, const Ctl& c, Unit& U) {
+  if constexpr (RING) return take_unit_warp(smem, sbase, it, c, U);
+  else return next_unit(p, it, U) ? 1 : 0;
+}
+// The same for a role run by one thread.
+__device__ __forceinline__ int take_unit(const uint8_t* smem, uint32_t sbase, int it, const Ctl& c,
+                                         Unit& U) {
+  const int slot = it & (UNIT_RING - 1);
+  if (!wait_bar(bar_addr(sbase, BAR_UFULL + slot), (it / UNIT_RING) & 1, c)) return -1;
+  const int valid = read_unit(smem, slot, U);
+  mbar_arrive(bar_addr(sbase, BAR_UEMPTY + slot));
+  return valid;
+}
+template <bool RING>
+__device__ __forceinline__ int get_unit(const Params& p, const uint8_t* smem, uint32_t sbase, int it,
+                                        const Ctl& c, Unit& U) {
+  if constexpr (RING) return take_unit(smem, sbase, it, c, U);
+  else return next_unit(p, it, U) ? 1 : 0;
+}
+
 // ============================================================ TMA producer
+// One thread. Loads each unit's Q tiles and streams its K/V tiles through
+// the ring of stages. With the unit ring (d = 64) it also decodes each unit
+// and publishes it there before its loads, so every role sees the next unit
+// early. Q tile t of the k-th unit that uses it goes to Q buffer k mod QBUF.
 template <int D, int MODE>
-__device__ void role_load(const Params& p, uint32_t sbase, const Ctl& c, const CUtensorMap* tm_q,
-                          const CUtensorMap* tm_k, const CUtensorMap* tm_v) {
+__device__ void role_load(const Params& p, uint8_t* smem, uint32_t sbase, const Ctl& c,
+                          const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v) {
   using L = Layout<D, MODE>;
-  constexpr bool BIAS = L::BIAS, FP8 = L::FP8;
-  (void)BIAS;
+  constexpr bool FP8 = L::FP8;
+  constexpr int QBUF = L::QBUF;
   (void)FP8;
-  uint32_t qe_ph[2] = {0, 0};
+  uint32_t qe_ph = 0;     // one bit per (tile, Q buffer)
+  int qcnt[2] = {0, 0};   // units that used each tile so far
   int st = 0;
   uint32_t kv_ph = 0;
   // parity of the last arming of each barrier, for the abort drain
-  uint32_t armed_q = 0, armed_kv = 0, last_q_ph[2] = {0, 0}, last_kv_ph[L::STAGES];
+  uint32_t armed_q = 0, armed_kv = 0, last_q_ph = 0, last_kv_ph[L::STAGES];
   bool ok = true;
   Unit U;
-  for (int it = 0; ok && next_unit(p, it, U); ++it) {
+  for (int it = 0; ok; ++it) {
+    const bool valid = next_unit(p, it, U);
+    if constexpr (L::RING) {
+      const int slot = it & (UNIT_RING - 1);
+      if (!(ok = wait_bar(bar_addr(sbase, BAR_UEMPTY + slot), ((it / UNIT_RING) & 1) ^ 1, c))) break;
+      write_unit(smem, slot, U, valid ? 1 : 0);
+      mbar_arrive(bar_addr(sbase, BAR_UFULL + slot));
+    }
+    if (!valid) break;
     for (int t = 0; t < 2 && ok; ++t) {
       if (!tile_active(U, t)) continue;
-      if (!(ok = wait_bar(bar_addr(sbase, BAR_QEMPTY + t), qe_ph[t] ^ 1, c))) break;
-      qe_ph[t] ^= 1;
-      const uint32_t full = bar_addr(sbase, BAR_QFULL + t);
+      const int qb = qcnt[t]++ & (QBUF - 1), qi = 2 * t + qb;
+      if (!(ok = wait_bar(bar_addr(sbase, BAR_QEMPTY + qi), ((qe_ph >> qi) & 1) ^ 1, c))) break;
+      qe_ph ^= 1u << qi;
+      const uint32_t full = bar_addr(sbase, BAR_QFULL + qi);
       mbar_arrive_expect_tx(full, L::Q_BYTES);
-      last_q_ph[t] = (armed_q >> t & 1) ? last_q_ph[t] ^ 1 : 0;
-      armed_q |= 1u << t;
+      last_q_ph = (armed_q >> qi & 1) ? last_q_ph ^ (1u << qi) : last_q_ph & ~(1u << qi);
+      armed_q |= 1u << qi;
       const int head = U.b * p.s.Hq + U.hq[t];
       // a 128-byte-wide box: 64 16-bit or 128 8-bit columns
       constexpr int BOX_COLS = 128 / L::ELEM;
       for (int bx = 0; bx < D / BOX_COLS; ++bx)
-        tma_load_3d(sbase + L::OFF_Q + t * L::Q_BYTES + bx * SW128_BOX_BYTES, tm_q, bx * BOX_COLS,
-                    U.mb[t] * BM, head, full);
+        tma_load_3d(sbase + L::OFF_Q + (qb * 2 + t) * L::Q_BYTES + bx * SW128_BOX_BYTES, tm_q,
+                    bx * BOX_COLS, U.mb[t] * BM, head, full);
     }
     const int kv_head = U.b * p.s.Hk + U.hk;
     for (int j = U.j0; j < U.nmax && ok; ++j) {
@@ -272,8 +361,8 @@ __device__ void role_load(const Params& p, uint32_t sbase, const Ctl& c, const C
     Ctl drain{c.abort_flag, 100000000ull};
     volatile int no_abort = 0;
     drain.abort_flag = &no_abort;
-    for (int t = 0; t < 2; ++t)
-      if (armed_q >> t & 1) wait_bar(bar_addr(sbase, BAR_QFULL + t), last_q_ph[t], drain);
+    for (int qi = 0; qi < 4; ++qi)
+      if (armed_q >> qi & 1) wait_bar(bar_addr(sbase, BAR_QFULL + qi), (last_q_ph >> qi) & 1, drain);
     for (int s = 0; s < L::STAGES; ++s)
       if (armed_kv >> s & 1) wait_bar(bar_addr(sbase, BAR_KV + s), last_kv_ph[s], drain);
   }
@@ -286,13 +375,18 @@ __device__ void role_load(const Params& p, uint32_t sbase, const Ctl& c, const C
 // the 128-byte swizzle, into the tile's single bias buffer. Rows and keys
 // past N read as zero (they are masked or never stored).
 template <int D>
-__device__ void role_bias_load(const Params& p, uint32_t sbase, const Ctl& c,
+__device__ void role_bias_load(const Params& p, const uint8_t* smem, uint32_t sbase, const Ctl& c,
                                const CUtensorMap* tm_b, int t) {
-  using L = Layout<D, true>;
+  using L = Layout<D, 1>;
   uint32_t be_ph = 0, last_ph = 0;
   bool armed = false, ok = true;
   Unit U;
-  for (int it = 0; ok && next_unit(p, it, U); ++it) {
+  for (int it = 0; ok; ++it) {
+    const int r = get_unit<Layout<D, 1>::RING>(p, smem, sbase, it, c, U);
+    if (r <= 0) {
+      ok = r == 0;
+      break;
+    }
     if (!tile_active(U, t)) continue;
     const int plane = U.b * p.bias_bmul * p.bias_H + U.hq[t] * p.bias_hmul;
     for (int j = U.j0; j < U.n[t] && ok; ++j) {
@@ -315,14 +409,250 @@ __device__ void role_bias_load(const Params& p, uint32_t sbase, const Ctl& c,
   }
 }
 
-// Run by the whole of warp 12, converged; one elected lane issues each
-// tcgen05 instruction.
+// Short-sequence form of the MMA warp (d = 64; see role_mma for the rest).
+// Per unit: S_t = Q_t·K_j0ᵀ for both tiles, then for every K/V tile j and
+// tile t: O_t += P_t·V_j (in two 64-key halves, the first as soon as the
+// softmax has stored half of P), then S_t for K_{j+1}. At a unit's last K/V
+// tile the first S of the NEXT unit (with work) is issued right behind each
+// tile's last P·V, so that tile's softmax restarts without waiting for the
+// other tile or for the epilogue: the next unit's K_j0 follows this unit's
+// last V_j in the ring of stages, its Q tiles were loaded into the other Q
+// buffers during this unit, and its P·V goes to the other O buffers.
 template <int D, bool BF16, int MODE>
-__device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const Ctl& c) {
+__device__ void role_mma_lookahead(const Params& p, const uint8_t* smem, uint32_t sbase,
+                                   uint32_t tmem, const Ctl& c) {
   using L = Layout<D, MODE>;
-  constexpr bool BIAS = L::BIAS, FP8 = L::FP8;
-  (void)BIAS;
+  constexpr bool FP8 = L::FP8;
+  static_assert(TmemO<D>::BUFS == 2 && L::QBUF == 2, "the look-ahead form double-buffers Q and O");
   (void)FP8;
+  // S = Q·Kᵀ, both K-major; O += P·V with V MN-major (16-bit) or, for FP8, Vᵀ
+  // K-major (E4M3 is format 0 of kind::f8f6f4, as fp16 is of kind::f16)
+  constexpr uint32_t IDESC_QK = idesc_f16(BF16 && !FP8, BN, false);
+  constexpr uint32_t IDESC_PV = idesc_f16(BF16 && !FP8, D, !FP8);
+  int st = 0;
+  uint32_t kv_ph = 0;
+  bool ok = true;
+
+  // Issue cost matters as much as tensor time here: one 128x128x16 MMA runs
+  // in ~64 cycles, so each issue must be a handful of instructions. The K
+  // loops are unrolled with compile-time offsets added to a descriptor built
+  // once per call (a K step adds its byte offset >> 4 to the start-address
+  // field, bits 0-13, with no carry out since shared memory is < 256 KB), and
+  // the accumulate flag is a compile-time constant except on the first step.
+  // The plain kernels keep only the descriptors' low words live: the 64-bit
+  // form spilled in this 80-register warp and ran 4-5 % slower. The bias and
+  // FP8 kernels keep the 64-bit form (no spill in FP8; in the bias kernel the
+  // low-word form timed 13 % slower).
+  using Desc = std::conditional_t<MODE == 0, uint32_t, uint64_t>;
+  const Desc q_desc0 = (Desc)sdesc(sbase + L::OFF_Q, 16, 1024);
+  const Desc kv_desc0 = (Desc)sdesc(sbase + L::OFF_KV, 16, 1024);
+  const Desc v_desc0 = FP8 ? kv_desc0 : (Desc)sdesc(sbase + L::OFF_KV, SW128_BOX_BYTES, 1024);
+  auto issue_qk = [&](int t, int kst, int qb) {
+    const Desc qd = q_desc0 + (Desc)(((qb * 2 + t) * L::Q_BYTES) >> 4);
+    const Desc kd = kv_desc0 + (Desc)((kst * L::KV_BYTES) >> 4);
+    const uint32_t d_s = tmem + S_COL[t];
+    if constexpr (FP8) {  // K = 32 bytes per MMA, all inside one 128-byte row
+      mma_ss<true>(d_s, qd, kd, IDESC_QK, 0u);
+#pragma unroll
+      for (int k = 1; k < D / 32; ++k) mma_ss<true>(d_s, qd + 2 * k, kd + 2 * k, IDESC_QK, 1u);
+      return;
+    }
+    mma_ss<false>(d_s, qd, kd, IDESC_QK, 0u);
+#pragma unroll
+    for (int k = 1; k < D / 16; ++k) {
+      const uint32_t off = ((k >> 2) * SW128_BOX_BYTES + (k & 3) * 32) >> 4;
+      mma_ss<false>(d_s, qd + off, kd + off, IDESC_QK, 1u);
+    }
+  };
+  // P·V over keys [64·h, 64·h + 64) of the tile (h = 0: first half, 1: second)
+  // into the O buffer at TMEM column o_col.
+  auto issue_pv_half = [&](int t, int vst, int h, uint32_t acc, uint32_t o_col) {
+    // P: 16 keys = 8 TMEM columns (two 16-bit values per column); V: 16 key
+    // rows of 128 bytes in each 64-column box, boxes SW128_BOX_BYTES apart.
+    const Desc vd = v_desc0 + (Desc)((vst * L::KV_BYTES) >> 4);
+    const uint32_t d_o = tmem + o_col;
+    const uint32_t a_p = tmem + S_COL[t];
+    if constexpr (FP8) {
+      // P: 32 keys = 8 TMEM columns (four E4M3 values per column); Vᵀ rows
+      // hold keys, 32 keys = 32 bytes of each 128-byte row
+#pragma unroll
+      for (int k = 2 * h; k < 2 * h + 2; ++k)
+        mma_ts<true>(d_o, a_p + k * 8, vd + 2 * k, IDESC_PV, k == 0 ? acc : 1u);
+      return;
+    }
+    const int k0 = h * (BN / 32);
+    mma_ts<false>(d_o, a_p + k0 * 8, vd + ((k0 * 16 * 128) >> 4), IDESC_PV, acc);
+#pragma unroll
+    for (int k = k0 + 1; k < k0 + BN / 32; ++k)
+      mma_ts<false>(d_o, a_p + k * 8, vd + ((k * 16 * 128) >> 4), IDESC_PV, 1u);
+  };
+
+  // Phase bits, one per barrier the MMA warp waits on; QF and OF: one per
+  // (tile, buffer).
+  constexpr uint32_t QF = 0, PF = 4, OC = 6, PH = 8, OF = 10;
+  uint32_t ph = 0;
+  auto wait_flip = [&](int bar, uint32_t bit, uint32_t invert) {
+    const bool r = wait_bar_warp(bar_addr(sbase, bar), ((ph >> bit) & 1u) ^ invert, c);
+    ph ^= 1u << bit;
+    return r;
+  };
+  // The MMA warp needs only the K/V ranges of a unit (tile t visits
+  // [j0, n_t); units without work are skipped, so max(n0, n1) > j0).
+  struct Range {
+    int j0, n0, n1;
+  };
+  int it = 0;
+  // Next unit with work (units whose tiles see no key are skipped: nothing
+  // is loaded for them). 1: found, 0: none left, -1: a wait gave up.
+  auto next_work = [&](Range& R) -> int {
+    while (true) {
+      Unit U;
+      const int r = take_unit_warp(smem, sbase, it++, c, U);
+      if (r <= 0) return r;
+      if (U.nmax > U.j0) {
+        R = Range{U.j0, U.n[0], U.n[1]};
+        return 1;
+      }
+    }
+  };
+  // Buffer parities, one bit per tile: bits 0-1 the Q buffer the next unit
+  // using the tile takes, 2-3 the current unit's Q buffers, 4-5 the next
+  // unit's, 6-7 the current unit's O buffers. Q tile t of the k-th unit that
+  // uses it sits in Q buffer k mod 2; O likewise.
+  uint32_t bufs = 0;
+  // First S of tile t of a unit from the K stage kst (already waited for),
+  // from Q buffer q.
+  auto first_s = [&](const Range& R, int t, int kst, int q) {
+    const int qi = 2 * t + q;
+    if (!wait_flip(BAR_QFULL + qi, QF + qi, 0)) return false;
+    tc_fence_after();
+    issue_qk(t, kst, q);
+    umma_commit_warp(bar_addr(sbase, BAR_SFULL + t));
+    if ((t ? R.n1 : R.n0) == R.j0 + 1) umma_commit_warp(bar_addr(sbase, BAR_QEMPTY + qi));
+    return true;
+  };
+  // Takes the next Q buffer of tile t: returns it, records it as the
+  // current (cur) or next unit's buffer, and flips the tile's parity.
+  auto take_q = [&](int t, bool cur) {
+    const int q = (bufs >> t) & 1;
+    const int sh = (cur ? 2 : 4) + t;
+    bufs = (bufs & ~(1u << sh)) | ((uint32_t)q << sh);
+    bufs ^= 1u << t;
+    return q;
+  };
+
+  Range U;
+  int r0 = next_work(U);
+  ok = r0 >= 0;
+  bool have = r0 > 0;
+  if (ok && have) {
+    const int k0 = st;
+    const uint32_t k0_ph = kv_ph;
+    if (++st == L::STAGES) { st = 0; kv_ph ^= 1; }
+    ok = wait_bar_warp(bar_addr(sbase, BAR_KV + k0), k0_ph, c);
+    if (ok) tc_fence_after();
+    for (int t = 0; t < 2 && ok; ++t)
+      if ((t ? U.n1 : U.n0) > U.j0) ok = first_s(U, t, k0, take_q(t, true));
+    if (ok) umma_commit_warp(bar_addr(sbase, BAR_KV + L::STAGES + k0));
+  }
+  while (ok && have) {
+    const int j0 = U.j0, nmax = U.n0 > U.n1 ? U.n0 : U.n1;
+    Range Un{0, 0, 0};
+    bool have_next = false;
+    for (int j = j0; j < nmax && ok; ++j) {
+      const int vs = st;
+      const uint32_t vs_ph = kv_ph;
+      if (++st == L::STAGES) { st = 0; kv_ph ^= 1; }
+      const bool last = j + 1 == nmax;
+      if (last) {
+        const int r = next_work(Un);
+        ok = r >= 0;
+        if (!ok) break;
+        have_next = r > 0;
+      }
+      // K stage of this unit's next tile, or of the next unit's first tile
+      int kn = -1;
+      uint32_t kn_ph = 0;
+      if (!last || have_next) {
+        kn = st;
+        kn_ph = kv_ph;
+        if (++st == L::STAGES) { st = 0; kv_ph ^= 1; }
+      }
+      if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_KV + vs), vs_ph, c))) break;
+      bool kn_ready = false;
+      auto need_kn = [&]() {
+        if (kn_ready) return true;
+        kn_ready = true;
+        const bool r = wait_bar_warp(bar_addr(sbase, BAR_KV + kn), kn_ph, c);
+        tc_fence_after();
+        return r;
+      };
+      for (int t = 0; t < 2; ++t) {
+        const int nt = t ? U.n1 : U.n0;
+        const int ob = (bufs >> (6 + t)) & 1, qb = (bufs >> (2 + t)) & 1;
+        if (j < nt) {
+          if (!(ok = wait_flip(BAR_PHALF + t, PH + t, 0))) break;
+          if (j > j0) {
+            if (!(ok = wait_flip(BAR_OCORR + t, OC + t, 0))) break;
+          } else {
+            if (!(ok = wait_flip(BAR_OFREE + 2 * t + ob, OF + 2 * t + ob, 1))) break;
+          }
+          tc_fence_after();
+          const uint32_t o_col = TmemO<D>::col(t, ob);
+          issue_pv_half(t, vs, 0, j > j0 ? 1u : 0u, o_col);
+          if (!(ok = wait_flip(BAR_PFULL + t, PF + t, 0))) break;
+          tc_fence_after();
+          issue_pv_half(t, vs, 1, 1u, o_col);
+          if (j == nt - 1) {
+            umma_commit_warp(bar_addr(sbase, BAR_PVDONE + 2 * t + ob));
+          } else {
+            if (!(ok = need_kn())) break;
+            issue_qk(t, kn, qb);
+            umma_commit_warp(bar_addr(sbase, BAR_SFULL + t));
+            if (j + 2 == nt) umma_commit_warp(bar_addr(sbase, BAR_QEMPTY + 2 * t + qb));
+          }
+        }
+        if (last && have_next && (t ? Un.n1 : Un.n0) > Un.j0) {
+          // the next unit's first S for this tile, right behind its last P·V
+          // (its Q tile loaded into the other Q buffer during this unit)
+          if (!(ok = need_kn())) break;
+          if (!(ok = first_s(Un, t, kn, take_q(t, false)))) break;
+        }
+      }
+      if (!ok) break;
+      umma_commit_warp(bar_addr(sbase, BAR_KV + L::STAGES + vs));
+      if (kn >= 0) umma_commit_warp(bar_addr(sbase, BAR_KV + L::STAGES + kn));
+    }
+    // this unit's tiles move to their other O buffer; the next unit's Q
+    // buffers become the current ones
+    bufs ^= (U.n0 > j0 ? 1u << 6 : 0u) | (U.n1 > j0 ? 1u << 7 : 0u);
+    bufs = (bufs & ~(3u << 2)) | (((bufs >> 4) & 3u) << 2);
+    U = Un;
+    have = have_next;
+  }
+  if (!ok) {
+    // Let every issued MMA finish before TMEM is released.
+    volatile int no_abort = 0;
+    Ctl drain{&no_abort, 100000000ull};
+    umma_commit_warp(bar_addr(sbase, BAR_DRAIN));
+    wait_bar_warp(bar_addr(sbase, BAR_DRAIN), 0, drain);
+  }
+}
+
+// Run by the whole of warp 12, converged; one elected lane issues each
+// tcgen05 instruction. Per unit: S_t = Q_t·K_j0ᵀ for both tiles, then for
+// every K/V tile j and tile t: O_t += P_t·V_j (in two 64-key halves, the
+// first as soon as the softmax has stored half of P), then S_t for K_{j+1}.
+template <int D, bool BF16, int MODE>
+__device__ void role_mma(const Params& p, const uint8_t* smem, uint32_t sbase, uint32_t tmem,
+                         const Ctl& c) {
+  using L = Layout<D, MODE>;
+  constexpr bool FP8 = L::FP8;
+  (void)FP8;
+  if constexpr (L::RING) {
+    role_mma_lookahead<D, BF16, MODE>(p, smem, sbase, tmem, c);
+    return;
+  }
   // S = Q·Kᵀ, both K-major; O += P·V with V MN-major (16-bit) or, for FP8, Vᵀ
   // K-major (E4M3 is format 0 of kind::f8f6f4, as fp16 is of kind::f16)
   constexpr uint32_t IDESC_QK = idesc_f16(BF16 && !FP8, BN, false);
@@ -367,7 +697,7 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
     // P: 16 keys = 8 TMEM columns (two 16-bit values per column); V: 16 key
     // rows of 128 bytes in each 64-column box, boxes SW128_BOX_BYTES apart.
     const Desc vd = v_desc0 + (Desc)((vst * L::KV_BYTES) >> 4);
-    const uint32_t d_o = tmem + TmemO<D>::col(t);
+    const uint32_t d_o = tmem + TmemO<D>::col(t, 0);
     const uint32_t a_p = tmem + S_COL[t];
     if constexpr (FP8) {
       // P: 32 keys = 8 TMEM columns (four E4M3 values per column); Vᵀ rows
@@ -401,7 +731,7 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
     if (++st == L::STAGES) { st = 0; kv_ph ^= 1; }
     if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_KV + k0), k0_ph, c))) break;
     if (n0 > j0 && !(ok = wait_flip(BAR_QFULL + 0, QF + 0, 0))) break;
-    if (n1 > j0 && !(ok = wait_flip(BAR_QFULL + 1, QF + 1, 0))) break;
+    if (n1 > j0 && !(ok = wait_flip(BAR_QFULL + 2, QF + 1, 0))) break;
     tc_fence_after();
     // Q_t is released (QEMPTY) as soon as the unit's last S_t MMA is issued,
     // so the next unit's Q tile loads while this unit's softmax and P·V run.
@@ -413,7 +743,7 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
     if (n1 > j0) {
       issue_qk(1, k0);
       umma_commit_warp(bar_addr(sbase, BAR_SFULL + 1));
-      if (n1 == j0 + 1) umma_commit_warp(bar_addr(sbase, BAR_QEMPTY + 1));
+      if (n1 == j0 + 1) umma_commit_warp(bar_addr(sbase, BAR_QEMPTY + 2));
     }
     umma_commit_warp(bar_addr(sbase, BAR_KV + L::STAGES + k0));
 
@@ -437,7 +767,7 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
         if (j > j0) {
           if (!(ok = wait_flip(BAR_OCORR + t, OC + t, 0))) break;
         } else {
-          if (!(ok = wait_flip(BAR_OFREE + t, OF + t, 1))) break;
+          if (!(ok = wait_flip(BAR_OFREE + 2 * t, OF + t, 1))) break;
         }
         tc_fence_after();
         issue_pv_half(t, vs, 0, j > j0 ? 1u : 0u);
@@ -445,7 +775,7 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
         tc_fence_after();
         issue_pv_half(t, vs, 1, 1u);
         if (j == nt - 1) {
-          umma_commit_warp(bar_addr(sbase, BAR_PVDONE + t));
+          umma_commit_warp(bar_addr(sbase, BAR_PVDONE + 2 * t));
         } else {
           if (!kn_ready) {
             if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_KV + kn), kn_ph, c))) break;
@@ -454,7 +784,7 @@ __device__ void role_mma(const Params& p, uint32_t sbase, uint32_t tmem, const C
           }
           issue_qk(t, kn);
           umma_commit_warp(bar_addr(sbase, BAR_SFULL + t));
-          if (j + 2 == nt) umma_commit_warp(bar_addr(sbase, BAR_QEMPTY + t));
+          if (j + 2 == nt) umma_commit_warp(bar_addr(sbase, BAR_QEMPTY + 2 * t));
         }
       }
       if (!ok) break;
@@ -683,7 +1013,7 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
   int units_done = 0;
   const uint8_t* brow = smem + L::OFF_BIAS + t * L::BIAS_BYTES + r * 128;
   Unit U;
-  for (int it = 0; next_unit(p, it, U); ++it) {
+  for (int it = 0; get_unit_warp<L::RING>(p, smem, sbase, it, c, U) > 0; ++it) {
     if (!tile_active(U, t)) continue;
     const int row = U.mb[t] * BM + r;
     // l_e: sum of the unrounded P (gives LSE). l_o normalises O: l_e plus,
@@ -755,13 +1085,16 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
       tc_fence_before();
       mbar_arrive(bar_addr(sbase, BAR_PFULL + t));
     }
-    // One barrier per stats buffer: buffer (k & 1) is rewritten only after
-    // the epilogue of unit k has read it (the next-but-one unit's first P·V
-    // waits for that epilogue to free O), so no barrier runs a phase ahead.
-    const int buf = units_done & 1;
+    // One barrier per stats buffer. The first S of unit k is issued after the
+    // first P·V of unit k - 1, which waited for the epilogue of unit
+    // k - 1 - BUFS to free its O buffer (that epilogue read its stats first);
+    // with NSTATS >= BUFS + 1 buffers, buffer k mod NSTATS is rewritten only
+    // after its previous contents were read, so no barrier runs a phase ahead.
+    constexpr int NSTATS = TmemO<D>::NSTATS;
+    const int buf = units_done & (NSTATS - 1);
     stats[(buf * 2 + t) * BM + r] = make_float4(m, l_o, l_e, 0.f);
     ++units_done;
-    mbar_arrive(bar_addr(sbase, BAR_STATS + 2 * t + buf));
+    mbar_arrive(bar_addr(sbase, BAR_STATS + 4 * t + buf));
   }
 }
 
@@ -790,12 +1123,20 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
   const uint32_t lane_base = (uint32_t)wl * 32;
   const float* alpha_all = reinterpret_cast<const float*>(smem + L::OFF_ALPHA);
   const float4* stats = reinterpret_cast<const float4*>(smem + L::OFF_STATS);
-  uint32_t af_ph[2] = {0, 0}, pv_ph[2] = {0, 0};
+  constexpr int OBUF = TmemO<D>::BUFS, NSTATS = TmemO<D>::NSTATS;
+  uint32_t af_ph[2] = {0, 0}, pv_ph = 0;  // pv_ph: one bit per (tile, O buffer)
   int units_done[2] = {0, 0};
   int ost = 0;  // staging buffer toggle (per warp)
   bool ok = true;
   Unit U;
-  for (int it = 0; ok && next_unit(p, it, U); ++it) {
+  for (int it = 0; ok; ++it) {
+    const int got = get_unit_warp<L::RING>(p, smem, sbase, it, c, U);
+    if (got <= 0) {
+      ok = got == 0;
+      break;
+    }
+    // O buffer of each tile for this unit (units with the tile active, mod OBUF)
+    const int obuf[2] = {units_done[0] & (OBUF - 1), units_done[1] & (OBUF - 1)};
     // ---- rescale O_t for every K/V tile after the first
     for (int j = U.j0 + 1; j < U.nmax && ok; ++j) {
       for (int t = 0; t < 2; ++t) {
@@ -805,7 +1146,7 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
         const float a = alpha_all[t * BM + r];
         if (__any_sync(0xffffffffu, a != 1.f)) {
           tc_fence_after();
-          const uint32_t t_o = tmem + (lane_base << 16) + TmemO<D>::col(t);
+          const uint32_t t_o = tmem + (lane_base << 16) + TmemO<D>::col(t, obuf[t]);
 #pragma unroll 1
           for (int q = 0; q < D / 32; ++q) {
             uint32_t o[32];
@@ -830,13 +1171,15 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
       const int head = U.b * p.s.Hq + U.hq[t];
       float inv_l = 0.f, lse = -INFINITY;
       const bool has = tile_active(U, t);
+      const int ob = obuf[t];
       if (has) {
-        const int k = units_done[t]++, buf = k & 1;
-        if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_STATS + 2 * t + buf), (k >> 1) & 1, c)))
+        const int k = units_done[t]++, buf = k & (NSTATS - 1);
+        if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_STATS + 4 * t + buf), (k / NSTATS) & 1, c)))
           break;
         const float4 ml = stats[(buf * 2 + t) * BM + r];
-        if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_PVDONE + t), pv_ph[t], c))) break;
-        pv_ph[t] ^= 1;
+        const int pb = 2 * t + ob;
+        if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_PVDONE + pb), (pv_ph >> pb) & 1, c))) break;
+        pv_ph ^= 1u << pb;
         tc_fence_after();
         if (ml.y > 0.f) {
           inv_l = __frcp_rn(ml.y);
@@ -845,7 +1188,7 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
         }
       }
       const int slab_row0 = U.mb[t] * BM + 32 * wl;
-      const uint32_t t_o = tmem + (lane_base << 16) + TmemO<D>::col(t);
+      const uint32_t t_o = tmem + (lane_base << 16) + TmemO<D>::col(t, ob);
       if (p.o_part != nullptr) {
         // Split-KV: this split's O (normalised by its own l) and LSE, fp32,
         // for the merge kernel; each thread writes its row's 128-byte chunks.
@@ -859,7 +1202,7 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
             reg_pin_x32(o);
             if (q == D / 32 - 1) {
               tc_fence_before();
-              mbar_arrive(bar_addr(sbase, BAR_OFREE + t));
+              mbar_arrive(bar_addr(sbase, BAR_OFREE + 2 * t + ob));
             }
           } else {
 #pragma unroll
@@ -885,7 +1228,7 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
           reg_pin_x32(o);
           if (q == D / 32 - 1) {
             tc_fence_before();
-            mbar_arrive(bar_addr(sbase, BAR_OFREE + t));
+            mbar_arrive(bar_addr(sbase, BAR_OFREE + 2 * t + ob));
           }
         } else {
 #pragma unroll
@@ -940,21 +1283,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
-      mbar_init(bar_addr(sbase, BAR_QFULL + t), 1);
-      mbar_init(bar_addr(sbase, BAR_QEMPTY + t), 1);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(bar_addr(sbase, BAR_QFULL + 2 * t + b), 1);
+        mbar_init(bar_addr(sbase, BAR_QEMPTY + 2 * t + b), 1);
+      }
       mbar_init(bar_addr(sbase, BAR_SFULL + t), 1);
       mbar_init(bar_addr(sbase, BAR_PFULL + t), BM);
       mbar_init(bar_addr(sbase, BAR_PHALF + t), BM);
       mbar_init(bar_addr(sbase, BAR_AFULL + t), BM);
       mbar_init(bar_addr(sbase, BAR_OCORR + t), BM);
-      mbar_init(bar_addr(sbase, BAR_PVDONE + t), 1);
-      mbar_init(bar_addr(sbase, BAR_OFREE + t), BM);
-      mbar_init(bar_addr(sbase, BAR_STATS + 2 * t), BM);
-      mbar_init(bar_addr(sbase, BAR_STATS + 2 * t + 1), BM);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(bar_addr(sbase, BAR_PVDONE + 2 * t + b), 1);
+        mbar_init(bar_addr(sbase, BAR_OFREE + 2 * t + b), BM);
+      }
+      for (int b = 0; b < 4; ++b) mbar_init(bar_addr(sbase, BAR_STATS + 4 * t + b), BM);
       mbar_init(bar_addr(sbase, BAR_BFULL + t), 1);
       mbar_init(bar_addr(sbase, BAR_BEMPTY + t), BM);
     }
     mbar_init(bar_addr(sbase, BAR_DRAIN), 1);
+    // unit records: one writer; one arrival per reading warp (MMA 1, softmax
+    // 8, correction 4, and the two bias loaders in bias mode)
+    for (int u = 0; u < UNIT_RING; ++u) {
+      mbar_init(bar_addr(sbase, BAR_UFULL + u), 1);
+      mbar_init(bar_addr(sbase, BAR_UEMPTY + u), BIAS ? 15 : 13);
+    }
     for (int s = 0; s < L::STAGES; ++s) {
       mbar_init(bar_addr(sbase, BAR_KV + s), 1);
       mbar_init(bar_addr(sbase, BAR_KV + L::STAGES + s), 1);
@@ -988,10 +1340,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     role_correction<D, BF16, MODE>(p, smem, sbase, tmem, ctl, &tm_o);
   } else {
     setmaxnreg_dec<80>();
-    if (warp == 12) role_mma<D, BF16, MODE>(p, sbase, tmem, ctl);
-    if (warp == 13 && lane == 0) role_load<D, MODE>(p, sbase, ctl, &tm_q, &tm_k, &tm_v);
+    if (warp == 12) role_mma<D, BF16, MODE>(p, smem, sbase, tmem, ctl);
+    if (warp == 13 && lane == 0) role_load<D, MODE>(p, smem, sbase, ctl, &tm_q, &tm_k, &tm_v);
     if constexpr (BIAS) {
-      if (warp >= 14 && lane == 0) role_bias_load<D>(p, sbase, ctl, &tm_b, warp - 14);
+      if (warp >= 14 && lane == 0) role_bias_load<D>(p, smem, sbase, ctl, &tm_b, warp - 14);
     }
     __syncwarp();
   }
