@@ -342,12 +342,6 @@ int fa_unit_for(int cta, int it, int grid);
  * FA_ERR_CUDA otherwise. Allocates 8 bytes of device memory for the result. */
 int fa_selftest_wait_timeout(int ms);
 
-/* Self test of the FMA-pipe exponential the softmax uses for part of its
- * 2^x values: writes 2^x[i] from it to y_fma[i] and from ex2.approx to
- * y_mufu[i], for n device floats; synchronises. Returns FA_OK or a negative
- * fa_status. */
-int fa_selftest_exp2(const float* x, float* y_fma, float* y_mufu, int n);
-
 /* Library version, major*10000 + minor*100 + patch. */
 int fa_version(void);
 

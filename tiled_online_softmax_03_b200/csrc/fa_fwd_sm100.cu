@@ -49,6 +49,11 @@ namespace fa {
 __device__ int g_fa_status;  // first device-side error of any launch (0 = none)
 
 constexpr int NUM_THREADS = 512;
+// Warp roles, by warpgroup of four warps (a warp reaches the TMEM lanes of
+// its quarter, warp % 4, so each per-row role takes a whole warpgroup; the
+// control warpgroup holds the MMA warp, the TMA warp and the bias loaders).
+constexpr int WG_SOFT0 = 0, WG_SOFT1 = 1, WG_CORR = 2, WG_CTRL = 3;
+constexpr int W_MMA = 4 * WG_CTRL, W_LOAD = 4 * WG_CTRL + 1;
 constexpr int TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: keep a stale max until it is 2^8 behind
 constexpr int SW128_BOX_BYTES = BM * 128;  // one 128-row box of 64 16-bit columns
@@ -815,34 +820,6 @@ __device__ __forceinline__ uint32_t round_pack(float lo, float hi) {
   }
 }
 
-// 2^y for a pair of fp32 values on the FMA pipe, relieving the MUFU pipe
-// (16 ex2 per clock per SM), which otherwise takes as long per K/V tile as
-// the tensor core at d = 128. Cody-Waite style reduction y = n + f with
-// n = round(y) (by adding 1.5·2^23, whose low mantissa bits then hold n) and
-// f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose coefficients minimise
-// the maximum relative error (Remez exchange, csrc/fit_exp2_poly.py: 7.5e-5,
-// below the 16-bit rounding that P gets next); 2^n is added to the exponent
-// field. Inputs are clamped to >= -126, where 2^y is far below any P that
-// survives 16-bit rounding next to the row's maximum.
-constexpr float EXP2_C0 = 9.999280572e-01f;
-constexpr float EXP2_C1 = 6.932609677e-01f;
-constexpr float EXP2_C2 = 2.426111251e-01f;
-constexpr float EXP2_C3 = 5.517166853e-02f;
-__device__ __forceinline__ uint64_t exp2_fma2(uint64_t y) {
-  const uint64_t yc = f2_pack(fmaxf(f2_lo(y), -126.f), fmaxf(f2_hi(y), -126.f));
-  const uint64_t t = fadd2(yc, f2_pack(12582912.f, 12582912.f));
-  const uint64_t n = fadd2(t, f2_pack(-12582912.f, -12582912.f));
-  const uint64_t f = ffma2(n, f2_pack(-1.f, -1.f), yc);
-  uint64_t q = ffma2(f2_pack(EXP2_C3, EXP2_C3), f, f2_pack(EXP2_C2, EXP2_C2));
-  q = ffma2(q, f, f2_pack(EXP2_C1, EXP2_C1));
-  q = ffma2(q, f, f2_pack(EXP2_C0, EXP2_C0));
-  const uint32_t r0 = (uint32_t)q + ((uint32_t)t << 23);
-  const uint32_t r1 = (uint32_t)(q >> 32) + ((uint32_t)(t >> 32) << 23);
-  return ((uint64_t)r1 << 32) | r0;
-}
-// One pair in every EXP2_FMA_EVERY takes the FMA-pipe exponential (unmasked tiles).
-constexpr int EXP2_FMA_EVERY = 1 << 30;  // off: slower than ex2.approx alone in this kernel
-
 // Row max of one S tile for this thread's row, in log2 units of the scaled
 // score. MASKED: keys c >= nvalid are masked, and s is rewritten in place to
 // s·scale·log2e (−inf where masked); otherwise s stays raw and the max of the
@@ -924,15 +901,7 @@ __device__ __forceinline__ float exp_store(const uint32_t (&s)[BN], float sl2, f
   for (int i = 0; i < BN / 2; ++i) {
     const uint64_t x = ((uint64_t)s[2 * i + 1] << 32) | s[2 * i];
     const uint64_t y = MASKED ? fadd2(x, nm2) : ffma2(x, k2, nm2);
-    float p0, p1;
-    if (!MASKED && i % EXP2_FMA_EVERY == EXP2_FMA_EVERY - 1) {
-      const uint64_t e = exp2_fma2(y);
-      p0 = f2_lo(e);
-      p1 = f2_hi(e);
-    } else {
-      p0 = ex2_approx(f2_lo(y));
-      p1 = ex2_approx(f2_hi(y));
-    }
+    const float p0 = ex2_approx(f2_lo(y)), p1 = ex2_approx(f2_hi(y));
     acc[i & 3] = fadd2(acc[i & 3], f2_pack(p0, p1));
     pk[i] = round_pack<BF16>(p0, p1);
     if (i == BN / 4 - 1) {
@@ -1314,11 +1283,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     *abort_flag = 0;
     mbar_init_fence();
   }
-  if (warp == 12) {
+  if (warp == W_MMA) {
     tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 13 && lane == 0) {
+  if (warp == W_LOAD && lane == 0) {
     tma_prefetch_map(&tm_q);
     tma_prefetch_map(&tm_k);
     tma_prefetch_map(&tm_v);
@@ -1332,25 +1301,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const Ctl ctl{abort_flag, p.timeout_ns};
 
   // Register split: 2×176 (softmax) + 80 (correction) + 80 (MMA, loads) = 4 × 128.
-  if (warp < 8) {
+  const int wg = warp >> 2;
+  if (wg == WG_SOFT0 || wg == WG_SOFT1) {
     setmaxnreg_inc<176>();
-    role_softmax<D, BF16, MODE>(p, smem, sbase, tmem, ctl, warp >> 2);
-  } else if (warp < 12) {
+    role_softmax<D, BF16, MODE>(p, smem, sbase, tmem, ctl, wg == WG_SOFT0 ? 0 : 1);
+  } else if (wg == WG_CORR) {
     setmaxnreg_dec<80>();
     role_correction<D, BF16, MODE>(p, smem, sbase, tmem, ctl, &tm_o);
   } else {
     setmaxnreg_dec<80>();
-    if (warp == 12) role_mma<D, BF16, MODE>(p, smem, sbase, tmem, ctl);
-    if (warp == 13 && lane == 0) role_load<D, MODE>(p, smem, sbase, ctl, &tm_q, &tm_k, &tm_v);
+    if (warp == W_MMA) role_mma<D, BF16, MODE>(p, smem, sbase, tmem, ctl);
+    if (warp == W_LOAD && lane == 0) role_load<D, MODE>(p, smem, sbase, ctl, &tm_q, &tm_k, &tm_v);
     if constexpr (BIAS) {
-      if (warp >= 14 && lane == 0) role_bias_load<D>(p, smem, sbase, ctl, &tm_b, warp - 14);
+      if ((warp & 3) >= 2 && lane == 0)
+        role_bias_load<D>(p, smem, sbase, ctl, &tm_b, (warp & 3) - 2);
     }
     __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 12) {
+  if (warp == W_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -1440,22 +1411,6 @@ __global__ void __launch_bounds__(256) fa_transpose_u8_kernel(const uint8_t* __r
   for (int i = threadIdx.x; i < 64 * 64; i += blockDim.x) {
     const int r = i / 64, cidx = i % 64;  // r: d, cidx: key
     if (n0 + cidx < N) dst[(long long)(d0 + r) * N + n0 + cidx] = tile[cidx][r];
-  }
-}
-
-// Evaluates the FMA-pipe exponential and ex2.approx on n inputs.
-__global__ void fa_exp2_selftest_kernel(const float* x, float* y_fma, float* y_mufu, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i + 1 < n) {
-    const uint64_t e = exp2_fma2(f2_pack(x[i], x[i + 1]));
-    y_fma[i] = f2_lo(e);
-    y_fma[i + 1] = f2_hi(e);
-    y_mufu[i] = ex2_approx(x[i]);
-    y_mufu[i + 1] = ex2_approx(x[i + 1]);
-  } else if (i < n) {
-    const uint64_t e = exp2_fma2(f2_pack(x[i], 0.f));
-    y_fma[i] = f2_lo(e);
-    y_mufu[i] = ex2_approx(x[i]);
   }
 }
 
@@ -1925,19 +1880,6 @@ int fa_get_device_status(void) {
   if (cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(int)) != cudaSuccess)
     return fail(FA_ERR_CUDA, "clearing the status word failed");
   return status;
-}
-
-int fa_selftest_exp2(const float* x, float* y_fma, float* y_mufu, int n) {
-  if (n < 1) return fail(FA_ERR_INVALID_ARG, "n must be >= 1");
-  int rc;
-  if ((rc = check_range("x", x, (size_t)n * 4, 4)) != FA_OK) return rc;
-  if ((rc = check_range("y_fma", y_fma, (size_t)n * 4, 4)) != FA_OK) return rc;
-  if ((rc = check_range("y_mufu", y_mufu, (size_t)n * 4, 4)) != FA_OK) return rc;
-  const int pairs = (n + 1) / 2;
-  fa::fa_exp2_selftest_kernel<<<(pairs + 255) / 256, 256>>>(x, y_fma, y_mufu, n);
-  cudaError_t e = cudaDeviceSynchronize();
-  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "exp2 self test: %s", cudaGetErrorString(e));
-  return FA_OK;
 }
 
 // Runs the bounded wait on a barrier that nothing arrives at, with a limit of
