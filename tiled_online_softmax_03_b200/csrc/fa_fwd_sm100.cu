@@ -49,11 +49,7 @@ namespace fa {
 __device__ int g_fa_status;  // first device-side error of any launch (0 = none)
 
 constexpr int NUM_THREADS = 512;
-// Warp roles, by warpgroup of four warps (a warp reaches the TMEM lanes of
-// its quarter, warp % 4, so each per-row role takes a whole warpgroup; the
-// control warpgroup holds the MMA warp, the TMA warp and the bias loaders).
-constexpr int WG_SOFT0 = 0, WG_SOFT1 = 1, WG_CORR = 2, WG_CTRL = 3;
-constexpr int W_MMA = 4 * WG_CTRL, W_LOAD = 4 * WG_CTRL + 1;
+
 constexpr int TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: keep a stale max until it is 2^8 behind
 constexpr int SW128_BOX_BYTES = BM * 128;  // one 128-row box of 64 16-bit columns
@@ -1283,11 +1279,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     *abort_flag = 0;
     mbar_init_fence();
   }
-  if (warp == W_MMA) {
+  if (warp == 12) {
     tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == W_LOAD && lane == 0) {
+  if (warp == 13 && lane == 0) {
     tma_prefetch_map(&tm_q);
     tma_prefetch_map(&tm_k);
     tma_prefetch_map(&tm_v);
@@ -1301,27 +1297,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const Ctl ctl{abort_flag, p.timeout_ns};
 
   // Register split: 2×176 (softmax) + 80 (correction) + 80 (MMA, loads) = 4 × 128.
-  const int wg = warp >> 2;
-  if (wg == WG_SOFT0 || wg == WG_SOFT1) {
+  if (warp < 8) {
     setmaxnreg_inc<176>();
-    role_softmax<D, BF16, MODE>(p, smem, sbase, tmem, ctl, wg == WG_SOFT0 ? 0 : 1);
-  } else if (wg == WG_CORR) {
+    role_softmax<D, BF16, MODE>(p, smem, sbase, tmem, ctl, warp >> 2);
+  } else if (warp < 12) {
     setmaxnreg_dec<80>();
     role_correction<D, BF16, MODE>(p, smem, sbase, tmem, ctl, &tm_o);
   } else {
     setmaxnreg_dec<80>();
-    if (warp == W_MMA) role_mma<D, BF16, MODE>(p, smem, sbase, tmem, ctl);
-    if (warp == W_LOAD && lane == 0) role_load<D, MODE>(p, smem, sbase, ctl, &tm_q, &tm_k, &tm_v);
+    if (warp == 12) role_mma<D, BF16, MODE>(p, smem, sbase, tmem, ctl);
+    if (warp == 13 && lane == 0) role_load<D, MODE>(p, smem, sbase, ctl, &tm_q, &tm_k, &tm_v);
     if constexpr (BIAS) {
-      if ((warp & 3) >= 2 && lane == 0)
-        role_bias_load<D>(p, smem, sbase, ctl, &tm_b, (warp & 3) - 2);
+      if (warp >= 14 && lane == 0) role_bias_load<D>(p, smem, sbase, ctl, &tm_b, warp - 14);
     }
     __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == W_MMA) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
