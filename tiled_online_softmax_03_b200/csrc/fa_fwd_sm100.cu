@@ -14,15 +14,17 @@
 // (fa_schedule.cuh). Warp roles:
 //   warps 0-3   softmax for Q tile 0 (thread r owns row r: TMEM lane r)
 //   warps 4-7   softmax for Q tile 1
-//   warps 8-11  correction (rescale O in TMEM) and epilogue (O/l, LSE, stores)
+//   warps 8-11  correction (rescale O in TMEM at d = 128 with 16-bit inputs)
+//               and epilogue (O/l, LSE, stores)
 //   warp 12     tcgen05.mma issue (one thread)
 //   warp 13     TMA loads (one thread)
 //   warps 14-15 bias mode: TMA loads of the bias tiles of Q tile 0 / 1
 //                (one thread each); otherwise no work
 // Per K/V tile j and Q tile t the MMA thread issues S_t = Q_t·K_jᵀ into TMEM,
 // the softmax warps turn S_t into P_t (16-bit, written over S_t in TMEM) and
-// the running statistics, the correction warps rescale O_t, and the MMA thread
-// issues O_t += P_t·V_j with P read from TMEM. The two Q tiles alternate, so
+// the running statistics, O_t is rescaled when a row's reference max moved
+// (by the correction warps, or by the softmax warps themselves at d = 64 and
+// in FP8), and the MMA thread issues O_t += P_t·V_j with P read from TMEM. The two Q tiles alternate, so
 // the tensor core works on one tile while the other tile's softmax runs.
 //
 // Pipelines use mbarriers; every wait is bounded (globaltimer) and a wait that
@@ -85,8 +87,8 @@ enum {
   BAR_QEMPTY = 4,   // [2 tiles][2 Q buffers] MMA -> TMA: the unit's last QK no longer needs it
   BAR_SFULL = 8,    // [2] MMA -> softmax: S tile ready in TMEM
   BAR_PFULL = 10,   // [2] softmax -> MMA: P written to TMEM
-  BAR_AFULL = 12,   // [2] softmax -> correction: rescale factors in smem
-  BAR_OCORR = 14,   // [2] correction -> MMA: O rescaled
+  BAR_AFULL = 12,   // [2] softmax -> correction: rescale factors in smem (d = 128 bf16/fp16)
+  BAR_OCORR = 14,   // [2] correction -> MMA: O rescaled (d = 128 bf16/fp16)
   BAR_PVDONE = 16,  // [2 tiles][2 O buffers] MMA -> epilogue: last P·V of the unit done
   BAR_OFREE = 20,   // [2 tiles][2 O buffers] epilogue -> MMA: O read out of TMEM
   BAR_STATS = 24,   // [2 tiles][4 buffers] softmax -> epilogue: final m, l in smem
@@ -108,6 +110,11 @@ struct Layout {
   static constexpr bool BIAS = MODE == 1, FP8 = MODE == 2;
   static constexpr int ELEM = FP8 ? 1 : 2;  // bytes per Q, K, V element
   static constexpr bool RING = TmemO<D>::SHORT;  // unit ring, early next-unit S
+  // Who rescales O when a row's reference max moves: the softmax warps
+  // themselves, before signalling half of P (d = 64 and FP8, measured faster),
+  // or the correction warps, which the MMA warp then waits for (d = 128 with
+  // 16-bit inputs: faster where rescales are frequent, as with peaked rows).
+  static constexpr bool SELF_RESCALE = TmemO<D>::SHORT || MODE == 2;
   static constexpr int QBUF = TmemO<D>::SHORT ? 2 : 1;
   static constexpr int Q_BYTES = BM * D * ELEM;
   static constexpr int KV_BYTES = BN * D * ELEM;
@@ -490,7 +497,7 @@ __device__ void role_mma_lookahead(const Params& p, const uint8_t* smem, uint32_
 
   // Phase bits, one per barrier the MMA warp waits on; QF and OF: one per
   // (tile, buffer).
-  constexpr uint32_t QF = 0, PF = 4, OC = 6, PH = 8, OF = 10;
+  constexpr uint32_t QF = 0, PF = 4, PH = 8, OF = 10;
   uint32_t ph = 0;
   auto wait_flip = [&](int bar, uint32_t bit, uint32_t invert) {
     const bool r = wait_bar_warp(bar_addr(sbase, bar), ((ph >> bit) & 1u) ^ invert, c);
@@ -593,11 +600,7 @@ __device__ void role_mma_lookahead(const Params& p, const uint8_t* smem, uint32_
         const int ob = (bufs >> (6 + t)) & 1, qb = (bufs >> (2 + t)) & 1;
         if (j < nt) {
           if (!(ok = wait_flip(BAR_PHALF + t, PH + t, 0))) break;
-          if (j > j0) {
-            if (!(ok = wait_flip(BAR_OCORR + t, OC + t, 0))) break;
-          } else {
-            if (!(ok = wait_flip(BAR_OFREE + 2 * t + ob, OF + 2 * t + ob, 1))) break;
-          }
+          if (j == j0 && !(ok = wait_flip(BAR_OFREE + 2 * t + ob, OF + 2 * t + ob, 1))) break;
           tc_fence_after();
           const uint32_t o_col = TmemO<D>::col(t, ob);
           issue_pv_half(t, vs, 0, j > j0 ? 1u : 0u, o_col);
@@ -766,7 +769,8 @@ __device__ void role_mma(const Params& p, const uint8_t* smem, uint32_t sbase, u
         if (j >= nt) continue;
         if (!(ok = wait_flip(BAR_PHALF + t, PH + t, 0))) break;
         if (j > j0) {
-          if (!(ok = wait_flip(BAR_OCORR + t, OC + t, 0))) break;
+          if constexpr (!L::SELF_RESCALE)
+            if (!(ok = wait_flip(BAR_OCORR + t, OC + t, 0))) break;
         } else {
           if (!(ok = wait_flip(BAR_OFREE + 2 * t, OF + t, 1))) break;
         }
@@ -883,13 +887,33 @@ __device__ __forceinline__ float row_max_bias(uint32_t (&s)[BN], float sl2, int 
   return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
 }
 
+// O ← α·O for this thread's row of O in TMEM (t_o: this warp's lanes), when
+// any row of the warp has α ≠ 1. The caller has waited for this step's S, so
+// the previous P·V into O is complete; its arrival on the half-P barrier,
+// which follows, lets the next P·V start.
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t t_o, float alpha) {
+  if (!__any_sync(0xffffffffu, alpha != 1.f)) return;
+#pragma unroll 1
+  for (int q = 0; q < D / 16; ++q) {  // 16 columns at a time: S is still half in registers
+    uint32_t o[16];
+    tmem_ld_x16(t_o + 16 * q, o);
+    tmem_wait_ld();
+    reg_pin_x16(o);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+    tmem_st_x16(t_o + 16 * q, o);
+  }
+}
+
 // P = exp2(s·scale·log2e − mref) for this thread's row, rounded to 16 bits and
 // written over S in TMEM in two 64-key halves (arriving on half_bar after the
-// first); returns the sum of the unrounded P. Scale-and-subtract and the sum
-// use packed fp32 pairs.
-template <bool BF16, bool MASKED>
+// first, and after rescaling O by alpha); returns the sum of the unrounded P.
+// Scale-and-subtract and the sum use packed fp32 pairs.
+template <int D, bool BF16, bool MASKED, bool RESCALE>
 __device__ __forceinline__ float exp_store(const uint32_t (&s)[BN], float sl2, float mref,
-                                           uint32_t t_p, uint32_t half_bar) {
+                                           uint32_t t_p, uint32_t half_bar, uint32_t t_o,
+                                           float alpha) {
   const uint64_t k2 = f2_pack(sl2, sl2), nm2 = f2_pack(-mref, -mref);
   uint64_t acc[4] = {0, 0, 0, 0};
   uint32_t pk[BN / 2];
@@ -904,6 +928,7 @@ __device__ __forceinline__ float exp_store(const uint32_t (&s)[BN], float sl2, f
       // First 64 keys: store and signal now, so the P·V MMA on them can
       // overlap the second half of the exponentials.
       tmem_st_x32(t_p, pk);
+      if constexpr (RESCALE) rescale_o<D>(t_o, alpha);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(half_bar);
@@ -919,9 +944,10 @@ __device__ __forceinline__ float exp_store(const uint32_t (&s)[BN], float sl2, f
 // columns per tile), first 64 keys stored and signalled early. Returns the sum
 // of the unrounded P (LSE) and, in *qsum, the sum of the rounded P — the exact
 // denominator of the P·V product the tensor core forms from them.
-template <bool MASKED>
+template <int D, bool MASKED>
 __device__ __forceinline__ float exp_store_f8(const uint32_t (&s)[BN], float sl2, float mref,
-                                              uint32_t t_p, uint32_t half_bar, float* qsum) {
+                                              uint32_t t_p, uint32_t half_bar, float* qsum,
+                                              uint32_t t_o, float alpha) {
   const uint64_t k2 = f2_pack(sl2, sl2), nm2 = f2_pack(-mref, -mref);
   uint64_t acc[2] = {0, 0}, accq[2] = {0, 0};
   uint32_t pk[BN / 4];
@@ -942,6 +968,7 @@ __device__ __forceinline__ float exp_store_f8(const uint32_t (&s)[BN], float sl2
     pk[w] = word;
     if (w == BN / 8 - 1) {
       tmem_st_x16(t_p, pk);
+      rescale_o<D>(t_o, alpha);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(half_bar);
@@ -971,8 +998,9 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
   const int r = threadIdx.x & 127;                           // row within the Q tile
   const uint32_t lane_base = (uint32_t)((threadIdx.x >> 5) & 3) * 32;
   const uint32_t t_s = tmem + (lane_base << 16) + S_COL[t];  // this warp's lanes of S_t / P_t
-  float* alpha_s = reinterpret_cast<float*>(smem + L::OFF_ALPHA) + t * BM;
   float4* stats = reinterpret_cast<float4*>(smem + L::OFF_STATS);
+  float* alpha_s = reinterpret_cast<float*>(smem + L::OFF_ALPHA) + t * BM;
+  (void)alpha_s;
   const float sl2 = p.scale_log2;
   uint32_t sf_ph = 0, bf_ph = 0;
   int units_done = 0;
@@ -981,6 +1009,9 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
   for (int it = 0; get_unit_warp<L::RING>(p, smem, sbase, it, c, U) > 0; ++it) {
     if (!tile_active(U, t)) continue;
     const int row = U.mb[t] * BM + r;
+    // this warp's lanes of the unit's O buffer (the k-th unit of the tile uses buffer k mod BUFS)
+    const uint32_t t_o =
+        tmem + (lane_base << 16) + TmemO<D>::col(t, units_done & (TmemO<D>::BUFS - 1));
     // l_e: sum of the unrounded P (gives LSE). l_o normalises O: l_e plus,
     // per K/V tile, the rounding error of that tile's largest P (the weight
     // that dominates a peaked row), so that O divides the P·V sum by a
@@ -1022,25 +1053,33 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
       // (log2) above it: O and l share the reference, so the result is
       // unchanged, P stays below 2^8 and the O rescale is skipped.
       const float m_new = (m_cand > m + RESCALE_THRESHOLD) ? m_cand : m;
+      // α rescales O before the P·V of this tile may start (in exp_store, or
+      // by the correction warps); the first tile of a unit starts O afresh
       float alpha = 1.f;
-      if (m_new != m) alpha = ex2_approx(m - m_new);
-      if (j > U.j0) {
-        alpha_s[r] = alpha;
-        mbar_arrive(bar_addr(sbase, BAR_AFULL + t));
+      if constexpr (L::SELF_RESCALE) {
+        if (m_new != m && j > U.j0) alpha = ex2_approx(m - m_new);
+      } else {
+        if (m_new != m) alpha = ex2_approx(m - m_new);
+        if (j > U.j0) {
+          alpha_s[r] = alpha;
+          mbar_arrive(bar_addr(sbase, BAR_AFULL + t));
+        }
       }
       m = m_new;
       const float mref = (m == -INFINITY) ? 0.f : m;
       const uint32_t half_bar = bar_addr(sbase, BAR_PHALF + t);
       if constexpr (FP8) {
         float qsum;
-        const float lsum = masked ? exp_store_f8<true>(s, sl2, mref, t_s, half_bar, &qsum)
-                                  : exp_store_f8<false>(s, sl2, mref, t_s, half_bar, &qsum);
+        const float lsum =
+            masked ? exp_store_f8<D, true>(s, sl2, mref, t_s, half_bar, &qsum, t_o, alpha)
+                   : exp_store_f8<D, false>(s, sl2, mref, t_s, half_bar, &qsum, t_o, alpha);
         tmem_wait_st();
         l_e = l_e * alpha + lsum;
         l_o = l_o * alpha + qsum;
       } else {
-        const float lsum = masked ? exp_store<BF16, true>(s, sl2, mref, t_s, half_bar)
-                                  : exp_store<BF16, false>(s, sl2, mref, t_s, half_bar);
+        constexpr bool RS = L::SELF_RESCALE;
+        const float lsum = masked ? exp_store<D, BF16, true, RS>(s, sl2, mref, t_s, half_bar, t_o, alpha)
+                                  : exp_store<D, BF16, false, RS>(s, sl2, mref, t_s, half_bar, t_o, alpha);
         const float pmax = ex2_approx(m_cand - mref);  // this tile's largest P
         const float delta = round16<BF16>(pmax) - pmax;
         tmem_wait_st();
@@ -1086,10 +1125,12 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
   const int wl = (threadIdx.x >> 5) & 3;  // warp within the group = 32-row slab
   const int lane = threadIdx.x & 31;
   const uint32_t lane_base = (uint32_t)wl * 32;
-  const float* alpha_all = reinterpret_cast<const float*>(smem + L::OFF_ALPHA);
   const float4* stats = reinterpret_cast<const float4*>(smem + L::OFF_STATS);
   constexpr int OBUF = TmemO<D>::BUFS, NSTATS = TmemO<D>::NSTATS;
+  const float* alpha_all = reinterpret_cast<const float*>(smem + L::OFF_ALPHA);
   uint32_t af_ph[2] = {0, 0}, pv_ph = 0;  // pv_ph: one bit per (tile, O buffer)
+  (void)alpha_all;
+  (void)af_ph;
   int units_done[2] = {0, 0};
   int ost = 0;  // staging buffer toggle (per warp)
   bool ok = true;
@@ -1102,33 +1143,35 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
     }
     // O buffer of each tile for this unit (units with the tile active, mod OBUF)
     const int obuf[2] = {units_done[0] & (OBUF - 1), units_done[1] & (OBUF - 1)};
-    // ---- rescale O_t for every K/V tile after the first
-    for (int j = U.j0 + 1; j < U.nmax && ok; ++j) {
-      for (int t = 0; t < 2; ++t) {
-        if (j >= U.n[t]) continue;
-        if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_AFULL + t), af_ph[t], c))) break;
-        af_ph[t] ^= 1;
-        const float a = alpha_all[t * BM + r];
-        if (__any_sync(0xffffffffu, a != 1.f)) {
-          tc_fence_after();
-          const uint32_t t_o = tmem + (lane_base << 16) + TmemO<D>::col(t, obuf[t]);
+    // ---- rescale O_t for every K/V tile after the first (when the softmax does not)
+    if constexpr (!L::SELF_RESCALE) {
+      for (int j = U.j0 + 1; j < U.nmax && ok; ++j) {
+        for (int t = 0; t < 2; ++t) {
+          if (j >= U.n[t]) continue;
+          if (!(ok = wait_bar_warp(bar_addr(sbase, BAR_AFULL + t), af_ph[t], c))) break;
+          af_ph[t] ^= 1;
+          const float a = alpha_all[t * BM + r];
+          if (__any_sync(0xffffffffu, a != 1.f)) {
+            tc_fence_after();
+            const uint32_t t_o = tmem + (lane_base << 16) + TmemO<D>::col(t, obuf[t]);
 #pragma unroll 1
-          for (int q = 0; q < D / 32; ++q) {
-            uint32_t o[32];
-            tmem_ld_x32(t_o + 32 * q, o);
-            tmem_wait_ld();
-            reg_pin_x32(o);
+            for (int q = 0; q < D / 32; ++q) {
+              uint32_t o[32];
+              tmem_ld_x32(t_o + 32 * q, o);
+              tmem_wait_ld();
+              reg_pin_x32(o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * a);
-            tmem_st_x32(t_o + 32 * q, o);
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * a);
+              tmem_st_x32(t_o + 32 * q, o);
+            }
+            tmem_wait_st();
           }
-          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar_addr(sbase, BAR_OCORR + t));
         }
-        tc_fence_before();
-        mbar_arrive(bar_addr(sbase, BAR_OCORR + t));
       }
+      if (!ok) break;
     }
-    if (!ok) break;
     // ---- epilogue: O / l -> 16-bit -> smem (64-byte swizzle) -> TMA store; LSE
     for (int t = 0; t < 2 && ok; ++t) {
       if (!U.present[t]) continue;
