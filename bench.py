@@ -407,12 +407,33 @@ def time_forward(w, dev, stream, steps, warmup, rank, local, world, barrier, ran
     kern = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     kern_avg = rank_max(sum(kern) / len(kern))
     total = rank_max(t_begin.elapsed_time(t_end)) if flush is None else kern_avg * steps
+    host_us = host_call_us(binding, w, q, k, v, o, lse, lens, stream)
     del q, k, v, o, lse, flush
     torch.cuda.empty_cache()
     return {"kernel_ms": kern_avg, "kernel_ms_median": rank_max(statistics.median(kern)),
             "ms_per_step": total / steps, "clocks": clocks.summary(), "device_status": status,
+            "host_us_per_call": host_us,
             "l2": "inputs larger than L2 (no flush)" if in_bytes(w) > 126e6 else
                   "L2 flushed between steps (256 MB write); kernel event times only"}
+
+
+def host_call_us(binding, w, q, k, v, o, lse, lens, stream, calls=50):
+    """Host time of one fa_fwd C call (argument checks, tensor-map encoding and
+    the launch; the kernels run asynchronously), called directly through ctypes
+    so no Python-side marshalling is counted; mean over `calls` calls."""
+    import ctypes
+    lib = binding.lib
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.Hq, w.Hk,
+            w.N, w.d, ctypes.c_float(w.scale), 1 if w.causal else 0,
+            lens.data_ptr() if lens is not None else None, stream.cuda_stream,
+            binding.FA_BF16 if w.dtype == "bf16" else binding.FA_FP16)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        lib.fa_fwd(*args)
+    t1 = time.perf_counter()
+    torch.cuda.synchronize()
+    return 1e6 * (t1 - t0) / calls
 
 
 def workload_entry(w, t, world, burst, sustained):
@@ -427,6 +448,7 @@ def workload_entry(w, t, world, burst, sustained):
             "frac_of_burst": achieved / burst,
             "frac_of_sustained": achieved / sustained if sustained else None,
             "algorithmic_gbps": algorithmic_bytes(w) / (t["kernel_ms"] * 1e-3) / 1e9,
+            "host_us_per_call": t.get("host_us_per_call"),
             "clocks": t["clocks"], "l2": t["l2"], "device_status": t["device_status"]}
 
 
@@ -669,6 +691,7 @@ def main():
     # ---- every other workload, timed the same way (plain forward runs only)
     per_wl = {}
     plain = pipelined and not args.shape and not args.no_per_workload
+    head_host_us = host_call_us(binding, w, q, k, v, o, lse, lens, stream) if plain else None
     if plain:
         del hq_, hk_, hv_, ho, hl
         for name in PER_WORKLOAD:
@@ -740,7 +763,7 @@ def main():
     if plain:
         head = {"kernel_ms": kern_avg, "kernel_ms_median": statistics.median(kern_ms),
                 "ms_per_step": ms_per_step, "clocks": clk, "device_status": status,
-                "l2": config["l2"]}
+                "l2": config["l2"], "host_us_per_call": head_host_us}
         line["per_workload"] = {name: workload_entry(WORKLOADS[name], head if name == w.name
                                                      else per_wl[name], world, burst,
                                                      sustained if f8 is None else None)
