@@ -13,6 +13,7 @@ SRC = os.path.join(PKG, "csrc", "fa_fwd_sm100.cu")
 DEPS = [SRC, os.path.join(PKG, "csrc", "fa_ptx.cuh"), os.path.join(PKG, "csrc", "fa_schedule.cuh"),
         os.path.join(PKG, "csrc", "fa_bwd_sm100.cuh"),
         os.path.join(PKG, "csrc", "fa_host_pipeline.cuh"),
+        os.path.join(PKG, "csrc", "fa_host.cuh"),
         os.path.join(ROOT, "include", "fa.h")]
 LIB = os.path.join(PKG, "libfa.so")
 
