@@ -92,42 +92,9 @@ int check_range(const char* name, const void* ptr, size_t bytes, size_t align) {
   return FA_OK;
 }
 
-// Encoded 3-D tensor maps of this thread's recent calls, reused when a call
-// asks for the same map again (same address, type, extents and box): a call
-// encodes up to five maps, which is a measurable part of its host time for
-// small problems. A map only describes memory; every call still checks its
-// buffers' allocations first, so a reused map never covers memory the call
-// was not given.
-struct MapKey {
-  const void* ptr;
-  int type, swizzle;
-  cuuint64_t dims[3];
-  cuuint32_t box[2];
-  bool operator==(const MapKey& o) const {
-    return ptr == o.ptr && type == o.type && swizzle == o.swizzle && dims[0] == o.dims[0] &&
-           dims[1] == o.dims[1] && dims[2] == o.dims[2] && box[0] == o.box[0] && box[1] == o.box[1];
-  }
-};
-constexpr int MAP_CACHE = 16;
-struct MapCache {
-  MapKey key[MAP_CACHE];
-  CUtensorMap map[MAP_CACHE];
-  bool used[MAP_CACHE] = {};
-  int next = 0;
-};
-thread_local MapCache t_maps;
-
 // Dense 3-D map [dims[2]][dims[1]][dims[0]] of `elem`-byte elements.
 int encode_map(CUtensorMap* map, const void* ptr, CUtensorMapDataType type, int elem,
                const cuuint64_t (&dims)[3], int box_cols, int box_rows, CUtensorMapSwizzle swz) {
-  const MapKey k{ptr, (int)type, (int)swz, {dims[0], dims[1], dims[2]},
-                 {(cuuint32_t)box_cols, (cuuint32_t)box_rows}};
-  MapCache& c = t_maps;
-  for (int i = 0; i < MAP_CACHE; ++i)
-    if (c.used[i] && c.key[i] == k) {
-      *map = c.map[i];
-      return FA_OK;
-    }
   const cuuint64_t strides[2] = {dims[0] * elem, dims[0] * elem * dims[1]};
   const cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
@@ -136,11 +103,6 @@ int encode_map(CUtensorMap* map, const void* ptr, CUtensorMapDataType type, int 
                                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-  const int i = c.next;
-  c.next = (c.next + 1) % MAP_CACHE;
-  c.key[i] = k;
-  c.map[i] = *map;
-  c.used[i] = true;
   return FA_OK;
 }
 
