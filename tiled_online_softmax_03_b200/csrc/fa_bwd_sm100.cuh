@@ -87,6 +87,7 @@ struct BParams {
   float scale_log2;   // scale·log2e
   float scale;
   unsigned long long timeout_ns;
+  int ng;             // head groups of the unit order (0: one group)
 };
 
 struct BUnit {
@@ -96,12 +97,35 @@ struct BUnit {
 // Unit u: key block n = u / (B·Hk) (causal: smallest n, the most query tiles,
 // first), (b, hk) = u % (B·Hk). Steps: every query head of the group × query
 // tiles m >= m_lo (m_lo = n when causal); none if the block holds no valid key.
+// With ng > 0 groups the (b, hk) heads are cut into ng near-equal groups and
+// the order above runs within one group after the other, so that the CTAs in
+// flight read the Q and dO tiles of a few heads, which stay in L2.
 __device__ __forceinline__ bool bwd_unit(const BParams& p, int it, BUnit& U) {
   const int u = unit_for(blockIdx.x, it, gridDim.x);
   if (u >= p.num_units) return false;
   const int bhk_count = p.B * p.Hk;
-  U.n = u / bhk_count;
-  const int bhk = u % bhk_count;
+  int bhk;
+  if (p.ng > 0) {
+    const int nkb = p.num_units / bhk_count;  // key blocks per head
+    const int base = bhk_count / p.ng, rem = bhk_count % p.ng;
+    const int big_units = (base + 1) * nkb;
+    int g, r, gh;
+    if (u < rem * big_units) {
+      g = u / big_units;
+      r = u - g * big_units;
+      gh = base + 1;
+    } else {
+      const int v = u - rem * big_units;
+      g = rem + v / (base * nkb);
+      r = v - (g - rem) * base * nkb;
+      gh = base;
+    }
+    U.n = r / gh;
+    bhk = g * base + (g < rem ? g : rem) + r % gh;
+  } else {
+    U.n = u / bhk_count;
+    bhk = u % bhk_count;
+  }
   U.b = bhk / p.Hk;
   U.hk = bhk % p.Hk;
   int L = p.N;

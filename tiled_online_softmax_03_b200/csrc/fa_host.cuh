@@ -61,6 +61,7 @@ struct DeviceInfo {
   bool init = false;
   bool sm100 = false;
   int sms = 0;
+  long long l2_bytes = 0;
   bool attr_set[9] = {false, false, false, false, false, false, false, false, false};
   bool bwd_attr_set[4] = {false, false, false, false};
 };
@@ -330,6 +331,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
         return fail(FA_ERR_CUDA, "cudaGetDeviceProperties failed");
       info.sm100 = prop.major == 10 && prop.minor == 0;
       info.sms = prop.multiProcessorCount;
+      info.l2_bytes = prop.l2CacheSize;
       info.init = true;
     }
   }
@@ -619,6 +621,7 @@ extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o
         return fail(FA_ERR_CUDA, "cudaGetDeviceProperties failed");
       info.sm100 = prop.major == 10 && prop.minor == 0;
       info.sms = prop.multiProcessorCount;
+      info.l2_bytes = prop.l2CacheSize;
       info.init = true;
     }
   }
@@ -658,6 +661,23 @@ extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o
   bp.Npad = bp.NM * 128;
   bp.causal = causal;
   bp.num_units = (int)units;
+  {
+    // Head groups of the unit order: about 12 CTAs on each (b, hk) head at a
+    // time, so that they share its Q and dO tiles in L2. Only causal problems
+    // of at least eight waves of units, each group at least four waves, and
+    // only when fewer than 12 CTAs per head are in flight without groups
+    // (more CTAs on one head's tiles contend for the same L2 lines).
+    bp.ng = 0;
+    const long long grid = bp.num_units < info.sms ? bp.num_units : info.sms;
+    const long long heads = heads_k, nkb = (N + 127) / 128;
+    const long long per_group = grid / 12 > 0 ? grid / 12 : 1;
+    if (causal && heads * nkb >= 8 * grid && heads > per_group) {
+      long long ng = (heads + per_group - 1) / per_group;
+      const long long min_heads = (4 * grid + nkb - 1) / nkb;
+      if (ng > heads / min_heads) ng = heads / min_heads;
+      bp.ng = ng > 1 ? (int)ng : 0;
+    }
+  }
   bp.key_pad_lens = key_pad_lens;
   uint8_t* wsb = reinterpret_cast<uint8_t*>(workspace);
   float* dqacc = reinterpret_cast<float*>(wsb + ws.dq_off);
@@ -731,6 +751,7 @@ extern "C" int fa_fwd_fp8(const void* q, const void* k, const void* v, float q_d
         return fail(FA_ERR_CUDA, "cudaGetDeviceProperties failed");
       info.sm100 = prop.major == 10 && prop.minor == 0;
       info.sms = prop.multiProcessorCount;
+      info.l2_bytes = prop.l2CacheSize;
       info.init = true;
     }
   }
