@@ -335,6 +335,32 @@ int fa_unit_kv_range(int B, int Hq, int Hk, int N, int causal, int num_splits, i
  * (may be >= fa_num_units, meaning that CTA is done). */
 int fa_unit_for(int cta, int it, int grid);
 
+/* Causal problems whose grid would have fewer than ~12 CTAs on each (b, hk)
+ * head at a time order their units by head groups instead: every level of one
+ * group, heaviest first, then the next group, so that about 12 CTAs share each
+ * head's K/V tiles in L2 (the query heads of the GQA page "深度探索Flash-
+ * Attention中GQA性能调优技术解析" read their shared K/V from cache, section
+ * PackGQA). fa_unit_groups returns the number of near-equal groups fa_fwd uses
+ * at head dimension d = 128 without a bias on a `grid`-CTA launch of a device
+ * with `l2_bytes` of L2: 0 (one group, the plain order) for non-causal
+ * problems, problems of fewer than eight waves of units, problems with enough
+ * CTAs per head, problems whose K and V (4·N·d bytes a head) fit in half of the
+ * L2 already and problems where a group's would not; each group holds at least
+ * four waves. < 0 on bad arguments. fa_unit_kv_range_grouped is
+ * fa_unit_kv_range with `groups` such groups (0 gives fa_unit_kv_range's
+ * order); the first B·Hk mod groups groups hold one head more than the others.
+ * Host only. */
+int fa_unit_groups(int B, int Hq, int Hk, int N, int d, int causal, int grid, long long l2_bytes);
+/* Unit taken by CTA `cta` of a `grid`-CTA launch on its iteration `it` under
+ * that order with `groups` >= 2 groups (causal only): the serpentine walk of
+ * fa_unit_for restarts in each group, so every group is dealt out evenly by
+ * itself. Returns num_units·num_splits once the CTA is done, < 0 on bad
+ * arguments. Host only. */
+int fa_unit_for_grouped(int B, int Hq, int Hk, int N, int causal, int num_splits, int groups,
+                        int cta, int it, int grid);
+int fa_unit_kv_range_grouped(int B, int Hq, int Hk, int N, int causal, int num_splits, int groups,
+                             int u, int key_len, int32_t* out);
+
 /* Self test of the bounded wait: launches one thread that waits on an
  * mbarrier nothing arrives at, with a limit of `ms` (1..10000) milliseconds,
  * on the legacy default stream, and synchronises. Returns FA_OK when the wait

@@ -218,3 +218,123 @@ def test_fp8_arguments_rejected_before_cuda():
     assert lib.fa_fwd_fp8(*args(128, 128, ws=0)) == -1 and "workspace" in binding.last_error()
     assert binding.lib.fa_fwd_fp8_workspace_bytes(1, 2, 4096, 128) == 2 * 4096 * 128
     assert binding.lib.fa_fwd_fp8_workspace_bytes(1, 2, 4096, 64) == 0
+
+
+# ------------------------------------------------ head-grouped causal order
+
+GROUP_SHAPES = [(4, 32, 8, 8192, 1, 148), (1, 32, 32, 4096, 1, 148), (4, 32, 1, 8192, 1, 148),
+                (1, 16, 16, 32768, 1, 148), (2, 4, 2, 300, 1, 148), (32, 16, 16, 512, 0, 148),
+                (3, 6, 6, 4096, 1, 16), (5, 4, 2, 2048, 1, 24), (1, 6, 2, 1000, 1, 1)]
+
+
+L2 = 126 << 20  # B200
+
+
+def test_group_policy_on_the_workloads():
+    # 8K GQA: 32 (b, hk) heads of 4 MiB K+V on 148 CTAs -> 12 heads (48 MiB) per group -> 3 groups
+    assert binding.unit_groups(4, 32, 8, 8192, 128, 1, 148, L2) == 3
+    # 32K: a group of 12 heads' K+V (192 MiB) would not stay in L2 either: one group
+    assert binding.unit_groups(1, 16, 16, 32768, 128, 1, 148, L2) == 0
+    # 16 heads at N = 8K fit in half of L2: no groups; 64 of them do not
+    assert binding.unit_groups(1, 16, 16, 8192, 128, 1, 148, L2) == 0
+    assert binding.unit_groups(4, 16, 16, 8192, 128, 1, 148, L2) == 3
+    # enough CTAs per head already, or too few units, or not causal: one group
+    assert binding.unit_groups(4, 32, 1, 8192, 128, 1, 148, L2) == 0
+    assert binding.unit_groups(1, 32, 32, 4096, 128, 1, 148, L2) == 0
+    assert binding.unit_groups(32, 16, 16, 512, 64, 0, 148, L2) == 0
+    assert binding.unit_groups(2, 4, 2, 300, 128, 1, 148, L2) == 0
+    with pytest.raises(binding.FaError):
+        binding.unit_groups(1, 3, 2, 128, 128, 1, 148, L2)
+
+
+@pytest.mark.parametrize("B,Hq,Hk,N,causal,grid", GROUP_SHAPES)
+def test_grouped_order_is_a_permutation_heaviest_first_per_group(B, Hq, Hk, N, causal, grid):
+    heads = B * Hk
+    nu = binding.num_units(B, Hq, Hk, N, causal)
+    np_ = nu // heads
+    ngs = {binding.unit_groups(B, Hq, Hk, N, 128, causal, grid, L2)} | ({2, min(5, heads)} if causal else set())
+    for ng in sorted(ngs):
+        plain = {tuple(binding.unit_info(B, Hq, Hk, N, causal, u)) for u in range(nu)}
+        got = [binding.unit_kv_range_grouped(B, Hq, Hk, N, causal, 1, ng, u, N) for u in range(nu)]
+        assert {tuple(r[:8]) for r in got} == plain  # same units, each once
+        if ng < 2 or not causal:
+            assert got == [binding.unit_kv_range(B, Hq, Hk, N, causal, 1, u, N) for u in range(nu)]
+            continue
+        # contiguous groups of near-equal head counts, the larger groups first
+        base, rem = divmod(heads, ng)
+        u = 0
+        bhk_next = 0
+        for g in range(ng):
+            gh = base + (g < rem)
+            chunk = got[u:u + gh * np_]
+            members = sorted({r[0] * Hk + r[1] for r in chunk})
+            assert members == list(range(bhk_next, bhk_next + gh))
+            work = [max(r[3], r[6] if r[7] else 0) for r in chunk]
+            assert work == sorted(work, reverse=True)  # heaviest first within the group
+            u += gh * np_
+            bhk_next += gh
+        assert u == nu
+
+
+def test_grouped_ranges_match_the_plain_ones_per_unit():
+    B, Hq, Hk, N = 2, 6, 3, 1000
+    nu = binding.num_units(B, Hq, Hk, N, 1)
+    for splits in (1, 3):
+        plain = {}
+        for u in range(nu * splits):
+            r = binding.unit_kv_range(B, Hq, Hk, N, 1, splits, u, 700)
+            plain[(r[0], r[1], r[2], r[3], r[8])] = r
+        for u in range(nu * splits):
+            r = binding.unit_kv_range_grouped(B, Hq, Hk, N, 1, splits, 4, u, 700)
+            assert plain.pop((r[0], r[1], r[2], r[3], r[8])) == r
+        assert not plain
+    with pytest.raises(binding.FaError):
+        binding.unit_kv_range_grouped(B, Hq, Hk, N, 1, 1, B * Hk + 1, 0, N)
+
+
+@pytest.mark.parametrize("B,Hq,Hk,N,grid,groups,splits",
+                         [(4, 32, 8, 8192, 148, 3, 1), (4, 32, 8, 8192, 148, 2, 1),
+                          (1, 16, 16, 32768, 148, 2, 1), (3, 6, 6, 4096, 16, 4, 1),
+                          (5, 4, 2, 2048, 24, 3, 2), (2, 4, 2, 300, 7, 4, 3), (1, 6, 2, 1000, 1, 2, 1)])
+def test_grouped_assignment_partitions_each_group_in_turn(B, Hq, Hk, N, grid, groups, splits):
+    nu = binding.num_units(B, Hq, Hk, N, 1) * splits
+    heads = B * Hk
+    per_head = nu // heads
+    base, rem = divmod(heads, groups)
+    bounds = []  # first unit of each group
+    x = 0
+    for g in range(groups):
+        bounds.append(x)
+        x += (base + (g < rem)) * per_head
+    grid = min(grid, nu)
+    got = []
+    for cta in range(grid):
+        seq = []
+        it = 0
+        while True:
+            u = binding.unit_for_grouped(B, Hq, Hk, N, 1, splits, groups, cta, it, grid)
+            if u >= nu:
+                break
+            seq.append(u)
+            it += 1
+        gs = [max(i for i, b in enumerate(bounds) if b <= u) for u in seq]
+        assert gs == sorted(gs)  # groups in turn
+        assert seq == sorted(seq)  # and in list order (heaviest first) inside each group
+        got.extend(seq)
+    assert sorted(got) == list(range(nu))
+    # each group is dealt out by itself: its units go to the CTAs as evenly as possible
+    for g in range(groups):
+        lo = bounds[g]
+        hi = bounds[g + 1] if g + 1 < groups else nu
+        counts = {}
+        for cta in range(grid):
+            it = 0
+            while True:
+                u = binding.unit_for_grouped(B, Hq, Hk, N, 1, splits, groups, cta, it, grid)
+                if u >= nu:
+                    break
+                if lo <= u < hi:
+                    counts[cta] = counts.get(cta, 0) + 1
+                it += 1
+        c = [counts.get(cta, 0) for cta in range(grid)]
+        assert max(c) - min(c) <= 1 and sum(c) == hi - lo

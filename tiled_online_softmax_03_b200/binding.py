@@ -74,6 +74,12 @@ def load_library(path=LIB_PATH):
     L.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
     L.fa_unit_kv_range.argtypes = [c_int] * 8 + [ctypes.POINTER(ctypes.c_int32)]
     L.fa_unit_kv_range.restype = c_int
+    L.fa_unit_kv_range_grouped.argtypes = [c_int] * 9 + [ctypes.POINTER(ctypes.c_int32)]
+    L.fa_unit_kv_range_grouped.restype = c_int
+    L.fa_unit_for_grouped.argtypes = [c_int] * 10
+    L.fa_unit_for_grouped.restype = c_int
+    L.fa_unit_groups.argtypes = [c_int] * 7 + [ctypes.c_longlong]
+    L.fa_unit_groups.restype = c_int
     L.fa_last_error_string.argtypes = []
     L.fa_last_error_string.restype = ctypes.c_char_p
     L.fa_get_device_status.argtypes = []
@@ -445,3 +451,27 @@ def unit_kv_range(B, Hq, Hk, N, causal, num_splits, u, key_len):
     out = (ctypes.c_int32 * 12)()
     check(lib.fa_unit_kv_range(B, Hq, Hk, N, 1 if causal else 0, num_splits, u, key_len, out))
     return list(out)
+
+
+def unit_groups(B, Hq, Hk, N, d, causal, grid, l2_bytes):
+    """Head groups of the causal unit order fa_fwd uses at d = 128 (0: one group)."""
+    n = lib.fa_unit_groups(B, Hq, Hk, N, d, 1 if causal else 0, grid, l2_bytes)
+    if n < 0:
+        check(n)
+    return n
+
+
+def unit_kv_range_grouped(B, Hq, Hk, N, causal, num_splits, groups, u, key_len):
+    """unit_kv_range with the unit order cut into `groups` head groups."""
+    out = (ctypes.c_int32 * 12)()
+    check(lib.fa_unit_kv_range_grouped(B, Hq, Hk, N, 1 if causal else 0, num_splits, groups, u,
+                                       key_len, out))
+    return list(out)
+
+
+def unit_for_grouped(B, Hq, Hk, N, causal, num_splits, groups, cta, it, grid):
+    """Unit of CTA `cta` on iteration `it` under the grouped order (num_units·splits: done)."""
+    u = lib.fa_unit_for_grouped(B, Hq, Hk, N, 1 if causal else 0, num_splits, groups, cta, it, grid)
+    if u < 0:
+        check(u)
+    return u

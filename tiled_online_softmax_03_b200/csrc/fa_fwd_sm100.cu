@@ -104,10 +104,12 @@ enum {
 // Shared memory: barriers and flags first, then 1 KB-aligned tiles. With an
 // additive bias the K/V ring is halved to make room for one 128×128 16-bit
 // bias tile per Q tile.
-// MODE: 0 = plain, 1 = additive bias, 2 = FP8 (E4M3 Q, K, V).
+// MODE: 0 = plain, 1 = additive bias, 2 = FP8 (E4M3 Q, K, V), 3 = plain with
+// the head-grouped unit order (a kernel of its own, so that the others carry
+// no code for it).
 template <int D, int MODE = 0>
 struct Layout {
-  static constexpr bool BIAS = MODE == 1, FP8 = MODE == 2;
+  static constexpr bool BIAS = MODE == 1, FP8 = MODE == 2, GROUPED = MODE == 3;
   static constexpr int ELEM = FP8 ? 1 : 2;  // bytes per Q, K, V element
   static constexpr bool RING = TmemO<D>::SHORT;  // unit ring, early next-unit S
   // Who rescales O when a row's reference max moves: the softmax warps
@@ -229,11 +231,14 @@ __device__ __forceinline__ int key_len_of(const Params& p, int b) {
   return l < 0 ? 0 : (l > p.s.N ? p.s.N : l);
 }
 
-// Unit `it` of this CTA (serpentine order), decoded; false past the last one.
+// Unit `it` of this CTA (serpentine order, by head group in the grouped
+// kernel), decoded; false past the last one.
+template <bool GROUPED>
 __device__ __forceinline__ bool next_unit(const Params& p, int it, Unit& U) {
-  const int u = unit_for(blockIdx.x, it, gridDim.x);
+  const int u = GROUPED ? unit_for_grouped(p.s, blockIdx.x, it, gridDim.x)
+                        : unit_for(blockIdx.x, it, gridDim.x);
   if (u >= p.s.num_units) return false;
-  decode_unit(p.s, u, U);
+  decode_unit<GROUPED>(p.s, u, U);
   resolve_unit(p.s, key_len_of(p, U.b), U);
   return true;
 }
@@ -269,11 +274,11 @@ __device__ __forceinline__ int take_unit_warp(const uint8_t* smem, uint32_t sbas
   return valid;
 }
 // Unit `it` for a role: from the unit ring (RING), else decoded here.
-template <bool RING>
+template <bool RING, bool GROUPED>
 __device__ __forceinline__ int get_unit_warp(const Params& p, const uint8_t* smem, uint32_t sbase,
                                              int it, const Ctl& c, Unit& U) {
   if constexpr (RING) return take_unit_warp(smem, sbase, it, c, U);
-  else return next_unit(p, it, U) ? 1 : 0;
+  else return next_unit<GROUPED>(p, it, U) ? 1 : 0;
 }
 // The same for a role run by one thread.
 __device__ __forceinline__ int take_unit(const uint8_t* smem, uint32_t sbase, int it, const Ctl& c,
@@ -284,11 +289,11 @@ __device__ __forceinline__ int take_unit(const uint8_t* smem, uint32_t sbase, in
   mbar_arrive(bar_addr(sbase, BAR_UEMPTY + slot));
   return valid;
 }
-template <bool RING>
+template <bool RING, bool GROUPED>
 __device__ __forceinline__ int get_unit(const Params& p, const uint8_t* smem, uint32_t sbase, int it,
                                         const Ctl& c, Unit& U) {
   if constexpr (RING) return take_unit(smem, sbase, it, c, U);
-  else return next_unit(p, it, U) ? 1 : 0;
+  else return next_unit<GROUPED>(p, it, U) ? 1 : 0;
 }
 
 // ============================================================ TMA producer
@@ -312,7 +317,7 @@ __device__ void role_load(const Params& p, uint8_t* smem, uint32_t sbase, const 
   bool ok = true;
   Unit U;
   for (int it = 0; ok; ++it) {
-    const bool valid = next_unit(p, it, U);
+    const bool valid = next_unit<L::GROUPED>(p, it, U);
     if constexpr (L::RING) {
       const int slot = it & (UNIT_RING - 1);
       if (!(ok = wait_bar(bar_addr(sbase, BAR_UEMPTY + slot), ((it / UNIT_RING) & 1) ^ 1, c))) break;
@@ -390,7 +395,7 @@ __device__ void role_bias_load(const Params& p, const uint8_t* smem, uint32_t sb
   bool armed = false, ok = true;
   Unit U;
   for (int it = 0; ok; ++it) {
-    const int r = get_unit<Layout<D, 1>::RING>(p, smem, sbase, it, c, U);
+    const int r = get_unit<Layout<D, 1>::RING, false>(p, smem, sbase, it, c, U);
     if (r <= 0) {
       ok = r == 0;
       break;
@@ -451,7 +456,7 @@ __device__ void role_mma_lookahead(const Params& p, const uint8_t* smem, uint32_
   // form spilled in this 80-register warp and ran 4-5 % slower. The bias and
   // FP8 kernels keep the 64-bit form (no spill in FP8; in the bias kernel the
   // low-word form timed 13 % slower).
-  using Desc = std::conditional_t<MODE == 0, uint32_t, uint64_t>;
+  using Desc = std::conditional_t<MODE == 0 || MODE == 3, uint32_t, uint64_t>;
   const Desc q_desc0 = (Desc)sdesc(sbase + L::OFF_Q, 16, 1024);
   const Desc kv_desc0 = (Desc)sdesc(sbase + L::OFF_KV, 16, 1024);
   const Desc v_desc0 = FP8 ? kv_desc0 : (Desc)sdesc(sbase + L::OFF_KV, SW128_BOX_BYTES, 1024);
@@ -675,7 +680,7 @@ __device__ void role_mma(const Params& p, const uint8_t* smem, uint32_t sbase, u
   // form spilled in this 80-register warp and ran 4-5 % slower. The bias and
   // FP8 kernels keep the 64-bit form (no spill in FP8; in the bias kernel the
   // low-word form timed 13 % slower).
-  using Desc = std::conditional_t<MODE == 0, uint32_t, uint64_t>;
+  using Desc = std::conditional_t<MODE == 0 || MODE == 3, uint32_t, uint64_t>;
   const Desc q_desc0 = (Desc)sdesc(sbase + L::OFF_Q, 16, 1024);
   const Desc kv_desc0 = (Desc)sdesc(sbase + L::OFF_KV, 16, 1024);
   const Desc v_desc0 = FP8 ? kv_desc0 : (Desc)sdesc(sbase + L::OFF_KV, SW128_BOX_BYTES, 1024);
@@ -727,7 +732,7 @@ __device__ void role_mma(const Params& p, const uint8_t* smem, uint32_t sbase, u
     return r;
   };
   Unit U;
-  for (int it = 0; ok && next_unit(p, it, U); ++it) {
+  for (int it = 0; ok && next_unit<L::GROUPED>(p, it, U); ++it) {
     const int j0 = U.j0, n0 = U.n[0], n1 = U.n[1], nmax = U.nmax;
     if (nmax == j0) continue;
     const int k0 = st;
@@ -1006,7 +1011,7 @@ __device__ void role_softmax(const Params& p, uint8_t* smem, uint32_t sbase, uin
   int units_done = 0;
   const uint8_t* brow = smem + L::OFF_BIAS + t * L::BIAS_BYTES + r * 128;
   Unit U;
-  for (int it = 0; get_unit_warp<L::RING>(p, smem, sbase, it, c, U) > 0; ++it) {
+  for (int it = 0; get_unit_warp<L::RING, L::GROUPED>(p, smem, sbase, it, c, U) > 0; ++it) {
     if (!tile_active(U, t)) continue;
     const int row = U.mb[t] * BM + r;
     // this warp's lanes of the unit's O buffer (the k-th unit of the tile uses buffer k mod BUFS)
@@ -1136,7 +1141,7 @@ __device__ void role_correction(const Params& p, uint8_t* smem, uint32_t sbase, 
   bool ok = true;
   Unit U;
   for (int it = 0; ok; ++it) {
-    const int got = get_unit_warp<L::RING>(p, smem, sbase, it, c, U);
+    const int got = get_unit_warp<L::RING, L::GROUPED>(p, smem, sbase, it, c, U);
     if (got <= 0) {
       ok = got == 0;
       break;

@@ -62,7 +62,7 @@ struct DeviceInfo {
   bool sm100 = false;
   int sms = 0;
   long long l2_bytes = 0;
-  bool attr_set[9] = {false, false, false, false, false, false, false, false, false};
+  bool attr_set[11] = {};
   bool bwd_attr_set[4] = {false, false, false, false};
 };
 DeviceInfo g_dev[64];
@@ -244,6 +244,44 @@ int fa_unit_kv_range(int B, int Hq, int Hk, int N, int causal, int num_splits, i
 
 int fa_unit_for(int cta, int it, int grid) { return fa::unit_for(cta, it, grid); }
 
+int fa_unit_for_grouped(int B, int Hq, int Hk, int N, int causal, int num_splits, int groups,
+                        int cta, int it, int grid) {
+  const int nu = fa_num_units(B, Hq, Hk, N, causal);
+  if (nu < 0) return nu;
+  if (num_splits < 1 || num_splits > 16) return fail(FA_ERR_INVALID_ARG, "num_splits out of [1, 16]");
+  if (groups < 2 || groups > B * Hk || !causal)
+    return fail(FA_ERR_INVALID_ARG, "groups out of [2, B·Hk], or not causal");
+  if (grid < 1 || cta < 0 || cta >= grid || it < 0) return fail(FA_ERR_INVALID_ARG, "bad CTA or iteration");
+  fa::Shape s = fa::make_shape(B, Hq, Hk, N, causal, num_splits, groups);
+  fa::set_group_grid(s, grid);
+  return fa::unit_for_grouped(s, cta, it, grid);
+}
+
+int fa_unit_groups(int B, int Hq, int Hk, int N, int d, int causal, int grid, long long l2_bytes) {
+  if (B < 1 || Hq < 1 || Hk < 1 || N < 1 || Hq % Hk != 0 || grid < 1 || d < 1 || l2_bytes < 0)
+    return fail(FA_ERR_INVALID_ARG, "bad arguments");
+  return fa::group_count(B, Hq, Hk, N, causal, grid, 4LL * N * d, l2_bytes);
+}
+
+int fa_unit_kv_range_grouped(int B, int Hq, int Hk, int N, int causal, int num_splits, int groups,
+                             int u, int key_len, int32_t* out) {
+  const int nu = fa_num_units(B, Hq, Hk, N, causal);
+  if (nu < 0) return nu;
+  if (num_splits < 1 || num_splits > 16) return fail(FA_ERR_INVALID_ARG, "num_splits out of [1, 16]");
+  if (groups < 0 || groups > B * Hk) return fail(FA_ERR_INVALID_ARG, "groups out of [0, B·Hk]");
+  if (out == nullptr || u < 0 || (long long)u >= (long long)nu * num_splits)
+    return fail(FA_ERR_INVALID_ARG, "bad unit index");
+  if (key_len < 0 || key_len > N) return fail(FA_ERR_INVALID_ARG, "key_len out of [0, N]");
+  const fa::Shape s = fa::make_shape(B, Hq, Hk, N, causal, num_splits, groups);
+  fa::Unit U;
+  fa::decode_unit(s, u, U);
+  fa::resolve_unit(s, key_len, U);
+  const int32_t vals[12] = {U.b, U.hk, U.hq[0], U.mb[0], U.present[0], U.hq[1], U.mb[1],
+                            U.present[1], U.split, U.j0, U.n[0], U.n[1]};
+  memcpy(out, vals, sizeof(vals));
+  return FA_OK;
+}
+
 }  // extern "C"
 
 // ============================================ split-KV with a static scratch
@@ -402,7 +440,16 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     prm.lse_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
                                             (rows * d * 4 + 255) / 256 * 256);
   }
-  prm.s = fa::make_shape(B, Hq, Hk, N, causal, splits);
+  {
+    // head-grouped unit order (a kernel of its own: d = 128, no bias)
+    const fa::Shape s0 = fa::make_shape(B, Hq, Hk, N, causal, splits);
+    const int grid = s0.num_units < info.sms ? s0.num_units : info.sms;
+    const int ng = (d == 128 && bias == nullptr)
+                       ? fa::group_count(B, Hq, Hk, N, causal, grid, 4LL * N * d, info.l2_bytes)
+                       : 0;
+    prm.s = fa::make_shape(B, Hq, Hk, N, causal, splits, ng);
+    fa::set_group_grid(prm.s, grid);
+  }
   prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
   prm.timeout_ns = g_timeout_ns;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -415,6 +462,9 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     return bf16 ? launch<64, true, 1>(q, k, v, o, prm, st, info, 6, lse, bias, planes)
                 : launch<64, false, 1>(q, k, v, o, prm, st, info, 7, lse, bias, planes);
   }
+  if (d == 128 && prm.s.ng > 0)
+    return bf16 ? launch<128, true, 3>(q, k, v, o, prm, st, info, 9, lse)
+                : launch<128, false, 3>(q, k, v, o, prm, st, info, 10, lse);
   if (d == 128)
     return bf16 ? launch<128, true>(q, k, v, o, prm, st, info, 0, lse)
                 : launch<128, false>(q, k, v, o, prm, st, info, 1, lse);
