@@ -233,7 +233,9 @@ L2 = 126 << 20  # B200
 def test_group_policy_on_the_workloads():
     # 8K GQA: 32 (b, hk) heads of 4 MiB K+V on 148 CTAs -> 12 heads (48 MiB) per group -> 3 groups
     assert binding.unit_groups(4, 32, 8, 8192, 128, 1, 148, L2) == 3
-    # 32K: a group of 12 heads' K+V (192 MiB) would not stay in L2 either: one group
+    # the 32K workload: 8 (b, hk) heads, ~18 CTAs on each already: one group
+    assert binding.unit_groups(1, 32, 8, 32768, 128, 1, 148, L2) == 0
+    # 16 heads at 32K: a group of 12 heads' K+V (192 MiB) would not stay in L2 either: one group
     assert binding.unit_groups(1, 16, 16, 32768, 128, 1, 148, L2) == 0
     # 16 heads at N = 8K fit in half of L2: no groups; 64 of them do not
     assert binding.unit_groups(1, 16, 16, 8192, 128, 1, 148, L2) == 0
