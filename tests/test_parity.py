@@ -54,6 +54,16 @@ def test_head_groups(Hq, Hk, causal):
     check_full(w, x)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("N", [1000, 1024])
+def test_one_query_head_per_kv_head_several_units_per_cta(N, dtype):
+    # 40 heads × 4 tile pairs = 480 units on at most 148 CTAs: each CTA walks
+    # several units whose tile 0 ends one K/V tile before tile 1 (the next
+    # unit's first S is issued during that last tile)
+    w, x = small(3, 40, 40, N, 128, dtype, True, seed=N)
+    check_full(w, x)
+
+
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("d", [64, 128])
 def test_key_padding_edges(causal, d):
