@@ -173,6 +173,40 @@ def test_full_size_whole_head(name):
     _report(name, f"{len(picks)} tile-edge rows of (b={b2}, hq={h2})", errs, w.torch_dtype)
 
 
+@pytest.mark.parametrize("splits", [1, 2])
+def test_head_grouped_order_with_key_padding(splits):
+    """The 8K GQA shape runs the head-grouped unit order on a B200 (three
+    groups); here with per-sequence key lengths (full, ragged, one key, none)
+    and, with splits = 2, through split-KV, whose grouped order deals out
+    chunk pairs. Sampled rows and every row around the ragged length."""
+    from tiled_online_softmax_03_b200 import binding
+    w = WORKLOADS["gqa_8k_causal"]
+    props = torch.cuda.get_device_properties(0)
+    grid = min(binding.num_units(w.B, w.Hq, w.Hk, w.N, 1), props.multi_processor_count)
+    assert binding.unit_groups(w.B, w.Hq, w.Hk, w.N, w.d, 1, grid, props.L2_cache_size) > 1
+    x = make_inputs(w)
+    lens = torch.tensor([w.N, 5000, 1, 0], dtype=torch.int32)
+    dev = torch.device("cuda:0")
+    q, k, v, ld = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev), lens.to(dev)
+    if splits == 1:
+        o, lse = binding.fa_fwd(q, k, v, causal=True, scale=w.scale, key_pad_lens=ld)
+    else:
+        o, lse = binding.fa_fwd_splitkv(q, k, v, splits, causal=True, scale=w.scale, key_pad_lens=ld)
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    picks = set(sample_picks(w.B, w.Hq, w.N, 120, seed=w.seed + splits))
+    for i in (4990, 4999, 5000, 5001, 5119, 5120, w.N - 1):
+        picks.add((1, 3, i))
+    for i in (0, 1, 200, w.N - 1):
+        picks.update({(2, 7, i), (3, 30, i)})
+    picks = sorted(picks)
+    o_ref, lse_ref = oracle_rows(x["q"], x["k"], x["v"], True, w.scale, lens, picks)
+    idx = tuple(np.array(picks).T)
+    errs = compare(to64(o)[idx], to64(lse)[idx], o_ref, lse_ref, w.torch_dtype)
+    _report(w.name, f"key lengths {lens.tolist()}, splits {splits}: {len(picks)} rows", errs,
+            w.torch_dtype)
+
+
 def test_llama7b_4k_two_heads_full():
     w = WORKLOADS["llama7b_4k_causal"]
     x = make_inputs(w)
