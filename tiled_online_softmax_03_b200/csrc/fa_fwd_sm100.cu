@@ -470,6 +470,15 @@ __device__ void role_mma_lookahead(const Params& p, const uint8_t* smem, uint32_
       for (int k = 1; k < D / 32; ++k) mma_ss<true>(d_s, qd + 2 * k, kd + 2 * k, IDESC_QK, 1u);
       return;
     }
+    if constexpr (MODE == 0) {  // four MMAs per asm block (plain kernel; measured on the
+                                // grouped kernel without gain, which keeps one per block)
+      static_assert(D == 64 || D == 128, "head dim");
+      umma_ss_lo_x4<SDESC_HI, SDESC_HI, 2, 2>(d_s, qd, kd, IDESC_QK, 0u);
+      if constexpr (D == 128)
+        umma_ss_lo_x4<SDESC_HI, SDESC_HI, 2, 2>(d_s, qd + (SW128_BOX_BYTES >> 4),
+                                                 kd + (SW128_BOX_BYTES >> 4), IDESC_QK, 1u);
+      return;
+    }
     mma_ss<false>(d_s, qd, kd, IDESC_QK, 0u);
 #pragma unroll
     for (int k = 1; k < D / 16; ++k) {
@@ -494,6 +503,10 @@ __device__ void role_mma_lookahead(const Params& p, const uint8_t* smem, uint32_
       return;
     }
     const int k0 = h * (BN / 32);
+    if constexpr (MODE == 0) {  // one asm block (plain kernel)
+      umma_ts_lo_x4<SDESC_HI, 8, 128>(d_o, a_p + k0 * 8, vd + k0 * 128, IDESC_PV, acc);
+      return;
+    }
     mma_ts<false>(d_o, a_p + k0 * 8, vd + ((k0 * 16 * 128) >> 4), IDESC_PV, acc);
 #pragma unroll
     for (int k = k0 + 1; k < k0 + BN / 32; ++k)
@@ -694,6 +707,15 @@ __device__ void role_mma(const Params& p, const uint8_t* smem, uint32_t sbase, u
       for (int k = 1; k < D / 32; ++k) mma_ss<true>(d_s, qd + 2 * k, kd + 2 * k, IDESC_QK, 1u);
       return;
     }
+    if constexpr (MODE == 0) {  // four MMAs per asm block (plain kernel; measured on the
+                                // grouped kernel without gain, which keeps one per block)
+      static_assert(D == 64 || D == 128, "head dim");
+      umma_ss_lo_x4<SDESC_HI, SDESC_HI, 2, 2>(d_s, qd, kd, IDESC_QK, 0u);
+      if constexpr (D == 128)
+        umma_ss_lo_x4<SDESC_HI, SDESC_HI, 2, 2>(d_s, qd + (SW128_BOX_BYTES >> 4),
+                                                 kd + (SW128_BOX_BYTES >> 4), IDESC_QK, 1u);
+      return;
+    }
     mma_ss<false>(d_s, qd, kd, IDESC_QK, 0u);
 #pragma unroll
     for (int k = 1; k < D / 16; ++k) {
@@ -717,6 +739,10 @@ __device__ void role_mma(const Params& p, const uint8_t* smem, uint32_t sbase, u
       return;
     }
     const int k0 = h * (BN / 32);
+    if constexpr (MODE == 0) {  // one asm block (plain kernel)
+      umma_ts_lo_x4<SDESC_HI, 8, 128>(d_o, a_p + k0 * 8, vd + k0 * 128, IDESC_PV, acc);
+      return;
+    }
     mma_ts<false>(d_o, a_p + k0 * 8, vd + ((k0 * 16 * 128) >> 4), IDESC_PV, acc);
 #pragma unroll
     for (int k = k0 + 1; k < k0 + BN / 32; ++k)

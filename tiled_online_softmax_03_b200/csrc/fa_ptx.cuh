@@ -244,6 +244,53 @@ __device__ __forceinline__ void umma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uin
         : "memory");
   }
 }
+// Four kind::f16 MMAs into one accumulator from one asm block, issued by one
+// elected lane: MMA i (i = 0..3) adds i·A_STEP and i·B_STEP to the operands'
+// descriptor low words (shared-memory A) or to the TMEM column of A (the TS
+// form); the first accumulates when acc != 0, the other three always. One
+// election and no per-MMA predicate set-up, so the issuing warp spends a few
+// instructions per MMA.
+template <uint32_t A_HI, uint32_t B_HI, uint32_t A_STEP, uint32_t B_STEP>
+__device__ __forceinline__ void umma_ss_lo_x4(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                              uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, q;\n\t.reg .b32 a1, b1;\n\t.reg .b64 a, b;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 q, %3, %3;\n\t"
+      "mov.b64 a, {%1, %5};\n\tmov.b64 b, {%2, %6};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p;\n\t"
+      "add.u32 a1, %1, %7;\n\tadd.u32 b1, %2, %8;\n\t"
+      "mov.b64 a, {a1, %5};\n\tmov.b64 b, {b1, %6};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+      "add.u32 a1, %1, %9;\n\tadd.u32 b1, %2, %10;\n\t"
+      "mov.b64 a, {a1, %5};\n\tmov.b64 b, {b1, %6};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+      "add.u32 a1, %1, %11;\n\tadd.u32 b1, %2, %12;\n\t"
+      "mov.b64 a, {a1, %5};\n\tmov.b64 b, {b1, %6};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(acc), "r"(A_HI), "r"(B_HI), "n"(A_STEP), "n"(B_STEP),
+      "n"(2 * A_STEP), "n"(2 * B_STEP), "n"(3 * A_STEP), "n"(3 * B_STEP)
+      : "memory");
+}
+template <uint32_t B_HI, uint32_t A_STEP, uint32_t B_STEP>
+__device__ __forceinline__ void umma_ts_lo_x4(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                              uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, q;\n\t.reg .b32 a1, b1;\n\t.reg .b64 b;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 q, %3, %3;\n\t"
+      "mov.b64 b, {%2, %5};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b, %3, p;\n\t"
+      "add.u32 a1, %1, %6;\n\tadd.u32 b1, %2, %7;\n\tmov.b64 b, {b1, %5};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b, %3, q;\n\t"
+      "add.u32 a1, %1, %8;\n\tadd.u32 b1, %2, %9;\n\tmov.b64 b, {b1, %5};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b, %3, q;\n\t"
+      "add.u32 a1, %1, %10;\n\tadd.u32 b1, %2, %11;\n\tmov.b64 b, {b1, %5};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b, %3, q;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(acc), "r"(B_HI), "n"(A_STEP), "n"(B_STEP),
+      "n"(2 * A_STEP), "n"(2 * B_STEP), "n"(3 * A_STEP), "n"(3 * B_STEP)
+      : "memory");
+}
 // The same two MMA forms for 8-bit operands (kind::f8f6f4; K = 32 per
 // instruction; E4M3 is format 0 in the instruction descriptor's A/B fields).
 __device__ __forceinline__ void umma_ss_f8_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
